@@ -1,0 +1,426 @@
+"""Benchmark: fully quantized NVFP4 linear layers at Llama-7B shapes on B200.
+
+One step = forward + backward of the seven linear layers of a Llama-7B block
+at 32768 tokens (batch 64 x seq 512): QKVO 4 x (4096 <- 4096), gate/up
+2 x (11008 <- 4096), down 1 x (4096 <- 11008).  Per layer: quantize X
+(row-wise RTN for fprop, transposed SR for wgrad), quantize W (16x16 tiles,
+both orientations), fprop, quantize dY (row-wise and transposed, SR), dgrad,
+wgrad -- the calls fqt_linear_fwd / fqt_linear_bwd make, issued one by one
+through the public API so that each GEMM and quantizer is bracketed by CUDA
+events on the launching stream.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--fmt nvfp4|mxfp4] [--wgrad-rht]
+
+Prints ONE JSON line (rank 0).  value = 6 * sum(M N K) flops of all ranks /
+max-over-ranks device time.  Inputs are synthetic (seeded), resident in HBM
+and larger than L2 (126 MB) -- no L2 flush is needed between steps.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+M_TOKENS = 32768
+LAYERS = [("qkvo", 4096, 4096)] * 4 + [("gate_up", 11008, 4096)] * 2 + [("down", 4096, 11008)]
+METRIC = "NVFP4 linear fwd+bwd TFLOPS & % FP4 peak; quantizer GB/s & % HBM BW"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP4_PER_BF16 = 4.0          # nominal dense FP4 / dense BF16 tensor throughput (9 / 2.25 PF)
+# Algorithmic bytes per element of one quantize call producing row-wise and
+# transposed outputs with an in-kernel amax: amax read 2 B + encode read 2 B
+# + two outputs of (0.5 B codes + 1/16 B scales).
+Q_BYTES_PER_ELEM = 2 + 2 + 2 * (0.5 + 1 / 16)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks sampling (nvidia-smi during the timed region)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.dev = device_index
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 6:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[2:6]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+class Layer:
+    def __init__(self, F, name, N, K, cfg, src, device):
+        self.name, self.N, self.K, self.M = name, N, K, M_TOKENS
+        self.x = src["X"].to(device, non_blocking=False)
+        self.w = src["W"].to(device)
+        self.dy = src["dY"].to(device)
+        self.cfg = cfg
+        self.sv = F.Saved.empty(self.M, N, K, cfg, device=device, logical_scales=False)
+        self.y = torch.empty((self.M, N), dtype=torch.bfloat16, device=device)
+        self.dx = torch.empty((self.M, K), dtype=torch.bfloat16, device=device)
+        self.dw = torch.empty((N, K), dtype=torch.float32, device=device)
+
+
+def make_layers(F, cfg, device, seed):
+    import fqt_synth as S
+    cache = {}
+    layers = []
+    for name, N, K in LAYERS:
+        if (N, K) not in cache:
+            cache[(N, K)] = S.llama_linear(N, K, M=M_TOKENS, seed=seed)
+        layers.append(Layer(F, name, N, K, cfg, cache[(N, K)], device))
+    return layers, cache
+
+
+def qparams_for(cfg, which):
+    """The quantize requests fqt_linear_fwd / fqt_linear_bwd issue."""
+    rn, m = cfg.rht_n, cfg.rht_mask
+    if which == "x":
+        return dict(fmt=cfg.fmt, round=cfg.round_fwd, round_t=cfg.round_x_t,
+                    rht_n=rn if m & 1 else 0, rht_n_t=rn if m & 4 else 0, rht_seed=cfg.seed,
+                    sr_seed=cfg.seed, sr_stream=0, sr_stream_t=3)
+    if which == "w":
+        return dict(fmt=cfg.fmt, block=cfg.w_block, round=cfg.round_fwd, round_t=cfg.round_fwd,
+                    rht_n=rn if m & 1 else 0, rht_n_t=rn if m & 2 else 0, rht_seed=cfg.seed)
+    return dict(fmt=cfg.fmt, round=cfg.round_bwd, round_t=cfg.round_bwd,
+                rht_n=rn if m & 2 else 0, rht_n_t=rn if m & 4 else 0, rht_seed=cfg.seed,
+                sr_seed=cfg.seed, sr_stream=1, sr_stream_t=2)
+
+
+def plan(F, layers, ws):
+    """The calls of one step: (kind, units, thunk) -- the calls
+    fqt_linear_fwd / fqt_linear_bwd make for each layer."""
+    calls = []
+    for L in layers:
+        sv = L.sv
+        qx, qw, qd = (qparams_for(L.cfg, k) for k in ("x", "w", "dy"))
+        calls += [
+            ("quant", L.M * L.K, lambda L=L, sv=sv, q=qx: F.fp4_quantize(L.x, sv.xq, sv.xq_t, ws=ws, **q)),
+            ("quant", L.N * L.K, lambda L=L, sv=sv, q=qw: F.fp4_quantize(L.w, sv.wq, sv.wq_t, ws=ws, **q)),
+            ("gemm", 2 * L.M * L.N * L.K, lambda L=L, sv=sv: F.fp4_gemm(sv.xq, sv.wq, L.y, ws=ws)),
+            ("quant", L.M * L.N, lambda L=L, sv=sv, q=qd: F.fp4_quantize(L.dy, sv.dyq, sv.dyq_t, ws=ws, **q)),
+            ("gemm", 2 * L.M * L.N * L.K, lambda L=L, sv=sv: F.fp4_gemm(sv.dyq, sv.wq_t, L.dx, ws=ws)),
+            ("gemm", 2 * L.M * L.N * L.K, lambda L=L, sv=sv: F.fp4_gemm(sv.dyq_t, sv.xq_t, L.dw, ws=ws)),
+        ]
+    return calls
+
+
+def step(calls, events=None):
+    """One pass of the hot path; `events` (pre-created pairs) brackets each call."""
+    for i, (kind, units, fn) in enumerate(calls):
+        if events is not None:
+            events[i][0].record()
+            fn()
+            events[i][1].record()
+        else:
+            fn()
+
+
+def e2e_run(F, layers, cache, cfg, ws, steps, device):
+    """Same workload through fqt_linear_fwd / fqt_linear_bwd with HOST buffers:
+    every step copies X, W, dY in from pinned memory and Y, dX, dW out."""
+    host = {}
+    for (N, K), src in cache.items():
+        host[(N, K)] = {
+            "X": src["X"].pin_memory(), "W": src["W"].pin_memory(), "dY": src["dY"].pin_memory(),
+            "Y": torch.empty((M_TOKENS, N), dtype=torch.bfloat16).pin_memory(),
+            "dX": torch.empty((M_TOKENS, K), dtype=torch.bfloat16).pin_memory(),
+            "dW": torch.empty((N, K), dtype=torch.float32).pin_memory()}
+    h2d = d2h = 0
+
+    def one():
+        nonlocal h2d, d2h
+        for L in layers:
+            h = host[(L.N, L.K)]
+            L.x.copy_(h["X"], non_blocking=True)
+            L.w.copy_(h["W"], non_blocking=True)
+            L.dy.copy_(h["dY"], non_blocking=True)
+            F.fqt_linear_fwd(L.cfg, L.x, L.w, L.y, L.sv, ws)
+            F.fqt_linear_bwd(L.cfg, L.dy, L.sv, L.dx, L.dw, ws)
+            h["Y"].copy_(L.y, non_blocking=True)
+            h["dX"].copy_(L.dx, non_blocking=True)
+            h["dW"].copy_(L.dw, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    for L in layers:
+        h2d += (L.x.numel() + L.w.numel() + L.dy.numel()) * 2
+        d2h += L.y.numel() * 2 + L.dx.numel() * 2 + L.dw.numel() * 4
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(steps):
+        one()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    return ms, h2d, d2h
+
+
+def cpu_baseline(rows_sample: int = 512, cols_sample: int = 1024, seed: int = 0, cache=None):
+    """The oracle, as it stands, on a bounded sample of the same workload: for
+    each of the 7 layers the first `rows_sample` tokens and the first
+    `cols_sample` output features (X[:r], W[:c], dY[:r, :c]): NVFP4 quantize
+    of X, W, dY in both orientations, then the three GEMMs in float64.
+    Throughput in the metric's unit: 6 * r * c * K flops per second."""
+    import fqt_synth as S
+    import oracle as O
+    t_total = 0.0
+    flops = 0
+    seen = {}
+    cache = cache or {}
+    r, c = rows_sample, cols_sample
+    for name, N, K in LAYERS:
+        if (N, K) not in seen:
+            d = cache.get((N, K)) or S.llama_linear(N, K, M=M_TOKENS, seed=seed)
+            seen[(N, K)] = (S.as_f32(d["X"][:r]), S.as_f32(d["W"][:c]), S.as_f32(d["dY"][:r, :c]))
+        X, W, dY = seen[(N, K)]
+        T = lambda a: np.ascontiguousarray(a.T)
+        t0 = time.perf_counter()
+        qx = O.nvfp4_quantize_1d(X)
+        qxt = O.nvfp4_quantize_1d(T(X), "sr", sr_seed=seed, sr_stream=3)
+        qw = O.nvfp4_quantize_2d(W)
+        qwt = O.nvfp4_quantize_2d(T(W))
+        qd = O.nvfp4_quantize_1d(dY, "sr", sr_seed=seed, sr_stream=1)
+        qdt = O.nvfp4_quantize_1d(T(dY), "sr", sr_seed=seed, sr_stream=2)
+        deq = lambda q, b=(1, 16): O.dequantize(q["codes"], q["scales"], b)
+        O.gemm(deq(qx), deq(qw, (16, 16)), s_dec_a=qx["s_dec"], s_dec_b=qw["s_dec"])
+        O.gemm(deq(qd), deq(qwt, (16, 16)), s_dec_a=qd["s_dec"], s_dec_b=qwt["s_dec"])
+        O.gemm(deq(qdt), deq(qxt), s_dec_a=qdt["s_dec"], s_dec_b=qxt["s_dec"])
+        t_total += time.perf_counter() - t0
+        flops += 6 * r * c * K
+    return {"value": flops / t_total / 1e12, "unit": "TFLOP/s", "cores": O.num_threads(),
+            "kind": "oracle", "seconds": round(t_total, 2),
+            "sample": f"first {r} of {M_TOKENS} tokens x first {c} output features of each of "
+                      "the 7 layers: NVFP4 quantize (both orientations) + 3 float64 GEMMs"}
+
+
+def run_ours(args, rank, world, device):
+    import fp4_fully_quantized_b200 as F
+    F.load()
+    fmt = F.MXFP4 if args.fmt == "mxfp4" else F.NVFP4
+    cfg = F.linear_cfg(fmt, out_dtype=F.OUT_BF16, seed=args.seed)
+    if args.wgrad_rht and fmt == F.NVFP4:
+        cfg.rht_mask = F.RHT_WGRAD
+    layers, cache = make_layers(F, cfg, device, args.seed + rank)
+    ws = F.Workspace(device=device)
+    calls = plan(F, layers, ws)
+    for _ in range(args.warmup):
+        step(calls)
+    torch.cuda.synchronize()
+    if ws.status() != 0:
+        raise RuntimeError(f"device status {ws.status()} after warm-up")
+
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    evs = [[(mk(), mk()) for _ in calls] for _ in range(args.steps)]
+    launches0 = F.kernel_launches()
+    t0, t1 = mk(), mk()
+    with ClockSampler(device.index) as clk:
+        t0.record()
+        for i in range(args.steps):
+            step(calls, evs[i])
+        t1.record()
+        torch.cuda.synchronize()
+    launches = F.kernel_launches() - launches0
+    if world > 1:
+        torch.distributed.barrier()
+    ms = t0.elapsed_time(t1) / args.steps
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    assert ws.status() == 0, f"device status {ws.status()}"
+
+    ev = [(kind, units, a, b) for per in evs for (kind, units, _), (a, b) in zip(calls, per)]
+    flops_step = sum(6 * M_TOKENS * N * K for _, N, K in LAYERS)
+    gemm_ms = sum(a.elapsed_time(b) for k, u, a, b in ev if k == "gemm")
+    gemm_fl = sum(u for k, u, a, b in ev if k == "gemm")
+    gemm_n = sum(1 for k, *_ in ev if k == "gemm")
+    q_ms = sum(a.elapsed_time(b) for k, u, a, b in ev if k == "quant")
+    q_elems = sum(u for k, u, a, b in ev if k == "quant")
+    q_n = sum(1 for k, *_ in ev if k == "quant")
+    pk, pk_src = peaks()
+    fp4_peak = pk["bf16_tflops_sustained"] * FP4_PER_BF16
+    gemm_tflops = gemm_fl / (gemm_ms * 1e-3) / 1e12
+    q_gbs = q_elems * Q_BYTES_PER_ELEM / (q_ms * 1e-3) / 1e9
+
+    e2e = None
+    if not args.no_e2e:
+        e_ms, h2d, d2h = e2e_run(F, layers, cache, cfg, ws, args.e2e_steps, device)
+        e_ms_t = torch.tensor([e_ms], dtype=torch.float64, device=device)
+        if world > 1:
+            torch.distributed.all_reduce(e_ms_t, op=torch.distributed.ReduceOp.MAX)
+        e2e = {"value": round(world * flops_step / (float(e_ms_t.item()) * 1e-3) / 1e12, 2),
+               "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": round(float(e_ms_t.item()), 3),
+               "api": "fqt_linear_fwd + fqt_linear_bwd, host buffers"}
+
+    out = {
+        "metric": METRIC,
+        "value": round(world * flops_step / (ms_max * 1e-3) / 1e12, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_max, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp4(e2m1)+e4m3 scales, fp32 accumulate" if fmt == F.NVFP4 else
+                 "fp4(e2m1)+e8m0 scales, fp32 accumulate",
+        "data": "synthetic (seeded): X N(0,1) with 1% Student-t(3) channels, W N(0,0.02^2), "
+                "dY N(0,1e-6)",
+        "config": {"workload": "Llama-7B linear layers fwd+bwd (QKVO x4 4096x4096, gate/up x2 "
+                               "11008x4096, down 11008->4096), tokens 32768 (bs 64 x seq 512)",
+                   "format": args.fmt, "rounding": "RTN fwd, SR bwd/update" if fmt == F.NVFP4
+                   else "RTN fwd/bwd", "weights": "16x16 tiles" if fmt == F.NVFP4 else "1x32",
+                   "rht": {0: "off", 4: "wgrad 16-pt", 7: "all GEMMs 32-pt"}.get(cfg.rht_mask),
+                   "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}"},
+        "roofline": {"kernel": "fp4_gemm_kernel (tcgen05 block-scaled)", "bound": "tensor",
+                     "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1),
+                     "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4),
+                     "peak_source": f"{pk_src}: bf16 sustained x {FP4_PER_BF16:g} (nominal FP4/BF16)",
+                     "traffic": None, "launches": gemm_n,
+                     "avg_ms": round(gemm_ms / max(gemm_n, 1), 4),
+                     "share_of_step": round(gemm_ms / (ms_max * args.steps), 3)},
+        "quantizer": {"bound": "hbm", "achieved": round(q_gbs, 1), "peak": pk["hbm_gbs"],
+                      "unit": "GB/s", "frac": round(q_gbs / pk["hbm_gbs"], 4),
+                      "bytes_per_elem": Q_BYTES_PER_ELEM, "launches": q_n,
+                      "share_of_step": round(q_ms / (ms_max * args.steps), 3)},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    if e2e is not None:
+        out["e2e"] = e2e
+    return out, cache
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle as it stands, on bounded samples."""
+    steps = []
+    for _ in range(args.warmup):
+        cpu_baseline(args.ref_rows, args.ref_cols)
+    for _ in range(args.steps):
+        steps.append(cpu_baseline(args.ref_rows, args.ref_cols))
+    v = statistics.median(s["value"] for s in steps)
+    secs = sum(s["seconds"] for s in steps)
+    flops_step = sum(6 * M_TOKENS * N * K for _, N, K in LAYERS)
+    ms = flops_step / (v * 1e12) * 1e3
+    cb = dict(steps[-1])
+    cb["value"] = round(v, 6)
+    return {"metric": METRIC, "impl": "reference", "value": round(v, 6), "unit": "TFLOP/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 1), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic (seeded)",
+            "config": {"workload": "Llama-7B linear layers fwd+bwd, tokens 32768; each step a "
+                                   f"bounded sample of {args.ref_rows} tokens x {args.ref_cols} "
+                                   "output features per layer"},
+            "cpu_baseline": cb, "seconds_total": round(secs, 1),
+            "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--fmt", choices=["nvfp4", "mxfp4"], default="nvfp4")
+    ap.add_argument("--wgrad-rht", action="store_true")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-rows", type=int, default=512)
+    ap.add_argument("--ref-cols", type=int, default=1024)
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    out, cache = run_ours(args, rank, world, device)
+    if rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(args.ref_rows, args.ref_cols, args.seed, cache)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

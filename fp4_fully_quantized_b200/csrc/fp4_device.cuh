@@ -1,0 +1,206 @@
+// fp4_device.cuh -- device building blocks of the FP4 quantizers (sm_100a).
+//
+// Formats ("FP4", Robots Atlas, Components / Hyperparameters): E2M1 elements
+// (levels 0, 0.5, 1, 1.5, 2, 3, 4, 6), NVFP4 = 16-value blocks with an E4M3
+// scale and an FP32 tensor scale, MXFP4 = 32-value blocks with an E8M0 scale.
+//
+// Every floating-point step that decides a code is written with explicit
+// round-to-nearest intrinsics (__fmul_rn, __fadd_rn, __fdiv_rn) so that the
+// compiler cannot contract or reorder it; E2M1 and E4M3 round-to-nearest-even
+// use the hardware cvt instructions.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+
+namespace fp4dev {
+
+// ---------------------------------------------------------------------------
+// Philox4x32-10 (Salmon et al., SC'11), counter-based: draw i of a stream is
+// word (i mod 4) of philox(counter = (i/4 lo, i/4 hi, stream, 0),
+// key = (seed lo, seed hi)).
+// ---------------------------------------------------------------------------
+constexpr uint32_t kPhiloxM0 = 0xD2511F53u;
+constexpr uint32_t kPhiloxM1 = 0xCD9E8D57u;
+constexpr uint32_t kPhiloxW0 = 0x9E3779B9u;
+constexpr uint32_t kPhiloxW1 = 0xBB67AE85u;
+constexpr uint32_t kRhtStream = 0x48414441u;
+
+struct U4 { uint32_t x, y, z, w; };
+
+__host__ __device__ __forceinline__ U4 philox4x32_10(uint64_t ctr_lo64, uint32_t stream,
+                                                     uint64_t seed) {
+  uint32_t c0 = (uint32_t)ctr_lo64, c1 = (uint32_t)(ctr_lo64 >> 32), c2 = stream, c3 = 0;
+  uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+#ifdef __CUDA_ARCH__
+    uint32_t hi0 = __umulhi(kPhiloxM0, c0), lo0 = kPhiloxM0 * c0;
+    uint32_t hi1 = __umulhi(kPhiloxM1, c2), lo1 = kPhiloxM1 * c2;
+#else
+    uint64_t p0 = (uint64_t)kPhiloxM0 * c0, p1 = (uint64_t)kPhiloxM1 * c2;
+    uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+    uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+#endif
+    uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+    c0 = n0; c1 = lo1; c2 = n2; c3 = lo0;
+    k0 += kPhiloxW0; k1 += kPhiloxW1;
+  }
+  return U4{c0, c1, c2, c3};
+}
+
+// Bit mask of the Hadamard signs: bit j set <=> d_j = -1 (bit 31 of draw j).
+__host__ inline uint32_t rht_sign_mask(uint64_t seed, int n) {
+  uint32_t m = 0;
+  for (int j = 0; j < n; j += 4) {
+    U4 w = philox4x32_10((uint64_t)(j >> 2), kRhtStream, seed);
+    uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    for (int q = 0; q < 4 && j + q < n; ++q) m |= (ws[q] >> 31) << (j + q);
+  }
+  return m;
+}
+
+// ---------------------------------------------------------------------------
+// BF16 unpacking (exact widening).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* v) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// E2M1 round-to-nearest-even, saturating: 8 floats -> 8 packed codes (32
+// bits), element 2j in the low nibble of byte j.  cvt packs its first source
+// operand into the high nibble.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t e2m1x8_rn(const float* v) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
+      "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
+      : "=r"(out)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]),
+        "f"(v[7]));
+  return out;
+}
+
+// E2M1 stochastic rounding of one value with draw u: with lo <= |v| <= hi the
+// neighbouring levels (|v| clamped to 6), round up iff u < ceil(p * 2^32),
+// p = (|v| - lo) / (hi - lo).  Level gaps: 0.5 below 2, 1 in [2, 4), 2 in
+// [4, 6].  Returns the 4-bit code (sign kept, also for results of 0).
+__device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t u) {
+  const uint32_t sign = (__float_as_uint(v) >> 31) << 3;
+  float a = fminf(fabsf(v), 6.0f);
+  float gap_scale, lo;           // gap_scale = 2^32 / gap
+  uint32_t code_lo;
+  if (a < 2.0f) {
+    float f = floorf(__fmul_rn(a, 2.0f));
+    lo = __fmul_rn(f, 0.5f);
+    code_lo = (uint32_t)f;
+    gap_scale = 8589934592.0f;   // 2^33
+  } else if (a < 4.0f) {
+    float f = floorf(a);
+    lo = f;
+    code_lo = (uint32_t)f + 2u;
+    gap_scale = 4294967296.0f;   // 2^32
+  } else {
+    lo = (a < 6.0f) ? 4.0f : 6.0f;
+    code_lo = (a < 6.0f) ? 6u : 7u;
+    gap_scale = 2147483648.0f;   // 2^31
+  }
+  const float y = __fmul_rn(__fsub_rn(a, lo), gap_scale);   // exact, < 2^32
+  const unsigned long long T = __float2ull_ru(y);            // ceil, exact
+  const uint32_t up = ((unsigned long long)u < T) ? 1u : 0u;
+  return sign | (code_lo + up);
+}
+
+// ---------------------------------------------------------------------------
+// E4M3 (bias 7, max 448, subnormals down to 2^-9) round-to-nearest-even with
+// saturation for a non-negative scale, and its exact decode.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t e4m3_rn_sat(float t) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(t));
+  return (uint32_t)(r & 0xFFu);
+}
+
+__device__ __forceinline__ float e4m3_value(uint32_t c) {
+  const uint32_t e = (c >> 3) & 15u, m = c & 7u;
+  if (e == 0) return __fmul_rn((float)m, 0.001953125f);          // m * 2^-9
+  return __uint_as_float(((e + 120u) << 23) | (m << 20));        // 2^(e-7) (1 + m/8)
+}
+
+// E8M0 scale 2^-e as an exact float for e in [-127, 127].
+__device__ __forceinline__ float exp2_neg_exact(int e) {
+  const int x = -e;                          // result 2^x, x in [-127, 127]
+  if (x >= -126) return __uint_as_float((uint32_t)(x + 127) << 23);
+  return __uint_as_float(1u << 22);          // 2^-127 (subnormal)
+}
+
+// floor(log2 b) from the binary32 encoding, b finite and > 0.
+__device__ __forceinline__ int floor_log2_f32(float b) {
+  const uint32_t bits = __float_as_uint(b);
+  const int E = (int)((bits >> 23) & 0xFF);
+  if (E > 0) return E - 127;
+  return (31 - __clz(bits & 0x7FFFFF)) - 149;
+}
+
+// NVFP4 tensor scales from the amax: s_enc = RN(2688 / A) (largest finite
+// float on overflow), s_dec = RN(A / 2688); A = 0 gives 1 and 1.
+__device__ __forceinline__ void nvfp4_global_scales(float A, float& s_enc, float& s_dec) {
+  if (A == 0.0f) { s_enc = 1.0f; s_dec = 1.0f; return; }
+  float e = __fdiv_rn(2688.0f, A);
+  if (isinf(e)) e = 3.402823466e38f;
+  s_enc = e;
+  s_dec = __fdiv_rn(A, 2688.0f);
+}
+
+// Byte offset of scale (r, s) in the tensor-core scale layout: 512-byte atoms
+// of 128 rows x 4 blocks, atoms ordered row-block major; within an atom, row
+// r%32 owns 16 bytes holding rows r, r+32, r+64, r+96 (4 blocks each).
+__host__ __device__ __forceinline__ int64_t mma_sf_offset(int64_t r, int64_t s, int64_t S) {
+  return ((r >> 7) * (S >> 2) + (s >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (s & 3);
+}
+
+// ---------------------------------------------------------------------------
+// In-register Walsh-Hadamard butterflies on 8 values: strides 1, 2, 4,
+// (a, b) -> (a + b, a - b).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void wht8(float* v) {
+#pragma unroll
+  for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (j & h) continue;
+      const float a = v[j], b = v[j + h];
+      v[j] = __fadd_rn(a, b);
+      v[j + h] = __fsub_rn(a, b);
+    }
+  }
+}
+
+// Stride-h stage across threads: this thread holds chunk `mine` of 8 values
+// and the partner (lane ^ lane_xor) holds the chunk h = 8 * lane_xor away.
+// The lower chunk becomes a + b, the upper one a - b (a = lower, b = upper).
+__device__ __forceinline__ void wht_cross(float* v, int lane_xor, bool upper) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float p = __shfl_xor_sync(0xFFFFFFFFu, v[j], lane_xor);
+    v[j] = upper ? __fsub_rn(p, v[j]) : __fadd_rn(v[j], p);
+  }
+}
+
+}  // namespace fp4dev

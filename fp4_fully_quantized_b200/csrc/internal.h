@@ -1,0 +1,72 @@
+// internal.h -- launchers shared between the C-ABI layer and the kernels.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "fp4.h"
+
+namespace fp4impl {
+
+// Status block at the start of every workspace.
+struct DeviceStatus {
+  uint32_t code;         // first device-detected fp4_status, 0 = none
+  uint32_t where;        // kernel-specific detail (e.g. which wait expired)
+  uint32_t pad[62];
+};
+static_assert(sizeof(DeviceStatus) == 256, "status block is 256 bytes");
+
+int sm_count();
+
+// Counts kernel launches enqueued by this library (fp4_kernel_launches).
+void count_launches(uint64_t n);
+
+// Records `code` into the status word unless one is already set.
+__device__ __forceinline__ void set_status(uint32_t* status, uint32_t code, uint32_t where) {
+  if (status != nullptr && atomicCAS(status, 0u, code) == 0u) status[1] = where;
+}
+
+// --- quantizer launchers (quantize.cu) ------------------------------------
+struct RowQuantArgs {
+  const void* x; int64_t rows, cols, ld;
+  int fmt, round, rht_n; uint32_t rht_mask;
+  uint64_t sr_seed; uint32_t sr_stream;
+  const float* amax_src;   // NVFP4: amax to encode with
+  float* amax_out;         // NVFP4: written with *amax_src when != amax_src
+  float* s_dec;            // written (NVFP4: amax/2688; MXFP4: 1)
+  uint8_t* codes; uint8_t* scales; uint8_t* scales_mma;
+  uint32_t* status;
+};
+
+cudaError_t launch_amax_rows(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                             int rht_n, uint32_t rht_mask, float* amax, cudaStream_t s);
+cudaError_t launch_amax_cols(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                             int rht_n, uint32_t rht_mask, float* amax, cudaStream_t s);
+cudaError_t launch_quant_rows(const RowQuantArgs& a, cudaStream_t s);
+// Transposed output: the quantized operand is x^T ([cols, rows]); rows of x
+// are the blocked dimension.  Fields keep the meaning of RowQuantArgs with
+// rows/cols those of x.
+cudaError_t launch_quant_cols(const RowQuantArgs& a, cudaStream_t s);
+// NVFP4 16x16 tiles: W (codes/scales/scales_mma) and W^T (codes_t/...).
+struct Quant2DArgs {
+  const void* x; int64_t rows, cols, ld;
+  const float* amax_src; float* s_dec; float* s_dec_t; float* amax_out; float* amax_out_t;
+  uint8_t* codes; uint8_t* scales; uint8_t* scales_mma;
+  uint8_t* codes_t; uint8_t* scales_t; uint8_t* scales_mma_t;
+  uint32_t* status;
+};
+cudaError_t launch_quant_2d(const Quant2DArgs& a, cudaStream_t s);
+
+// --- GEMM (gemm_sm100.cu) -------------------------------------------------
+struct GemmArgs {
+  const uint8_t* a_codes; const uint8_t* a_sf; const float* a_sdec;
+  const uint8_t* b_codes; const uint8_t* b_sf; const float* b_sdec;
+  int64_t M, N, K;
+  int fmt;               // FP4_NVFP4 / FP4_MXFP4
+  float alpha;
+  void* c; int64_t ldc; int out_f32;
+  float* c_amax;
+  uint32_t* status;
+};
+fp4_status gemm_launch(const GemmArgs& g, cudaStream_t s);
+
+}  // namespace fp4impl

@@ -1,0 +1,536 @@
+// quantize.cu -- HBM-bound FP4 quantizers for sm_100a.
+//
+// NVFP4 ("FP4", Robots Atlas, How it works / Components "NVFP4"): 16-value
+// blocks, E4M3 block scale, FP32 tensor scale from the tensor amax.
+// MXFP4 (Components "MXFP4"): 32-value blocks, E8M0 power-of-two scale.
+// Rounding ("FP4 All the Way", Key points): round-to-nearest in the forward
+// pass, stochastic rounding (Philox draws) in the backward and update passes.
+// Optional block-wise random Hadamard transform before quantizing ("FP4",
+// How it works; "Quartet", Approach).
+//
+// Row-wise kernels: each thread owns one 16-byte load (8 BF16 values); the
+// 2 (NVFP4) or 4 (MXFP4) threads of a block are adjacent lanes and combine
+// their block max and cross-thread Hadamard stages with warp shuffles, so a
+// warp reads 512 contiguous bytes per load instruction.
+// Transposed kernels: a 64 x 64 tile is staged through shared memory; each
+// thread then owns 32 consecutive rows of one column (blocks run down x's
+// columns) and writes 16 bytes of codes of the transposed operand.
+#include <cfloat>
+#include <cstdint>
+
+#include "fp4_device.cuh"
+#include "internal.h"
+
+namespace fp4impl {
+using namespace fp4dev;
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr float kRht32Scale = 0.17677669227123260f;   // RN(1/sqrt(32)) = 0x3E3504F3
+
+template <int RHT_N>
+__device__ __forceinline__ float rht_scale() {
+  return RHT_N == 16 ? 0.25f : kRht32Scale;
+}
+
+// Rotates the 8 values of chunk `q` (chunk index within its Hadamard block)
+// held by this lane; lanes holding the other chunks of the block are the
+// adjacent lanes (lane ^ 1, lane ^ 2).
+template <int RHT_N>
+__device__ __forceinline__ void rht_chunk(float* v, uint32_t mask, int q) {
+  if constexpr (RHT_N > 0) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if ((mask >> (8 * q + i)) & 1u) v[i] = -v[i];
+    wht8(v);
+#pragma unroll
+    for (int lx = 1; lx < RHT_N / 8; lx <<= 1) wht_cross(v, lx, (q & lx) != 0);
+    const float c = rht_scale<RHT_N>();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], c);
+  }
+}
+
+__device__ __forceinline__ void block_amax_atomic(float m, float* amax) {
+  __shared__ float red[kThreads / 32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  if (l == 0) red[w] = m;
+  __syncthreads();
+  if (w == 0) {
+    m = (l < (int)(blockDim.x >> 5)) ? red[l] : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    // |x| has a clear sign bit, so integer order equals float order; NaN
+    // patterns sort above +Inf and survive the max.
+    if (l == 0) atomicMax(reinterpret_cast<unsigned int*>(amax), __float_as_uint(m));
+  }
+}
+
+// |v| max that keeps NaN (fmaxf would drop it).
+__device__ __forceinline__ float absmax_keep_nan(float m, float v) {
+  const uint32_t a = __float_as_uint(v) & 0x7FFFFFFFu;
+  return __uint_as_float(max(__float_as_uint(m), a));
+}
+
+// ---------------------------------------------------------------------------
+// Row-wise amax (optionally of the rotated values).
+// ---------------------------------------------------------------------------
+template <int RHT_N>
+__global__ void __launch_bounds__(kThreads)
+amax_rows_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+                 uint32_t rht_mask, float* amax) {
+  const int64_t cpr = cols >> 3, total = rows * cpr;
+  const int lane = threadIdx.x & 31;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  float m = 0.0f;
+  for (int64_t g0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x - lane); g0 < total;
+       g0 += stride) {
+    const int64_t g = g0 + lane;
+    float v[8];
+    if (g < total) {
+      const int64_t r = g / cpr, j = g - r * cpr;
+      bf16x8_to_f32(ld_nc_v4(x + r * ld + j * 8), v);
+      if constexpr (RHT_N > 0) rht_chunk<RHT_N>(v, rht_mask, (int)(j % (RHT_N / 8)));
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+      if constexpr (RHT_N > 0) rht_chunk<RHT_N>(v, rht_mask, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = absmax_keep_nan(m, v[i]);
+  }
+  block_amax_atomic(m, amax);
+}
+
+// ---------------------------------------------------------------------------
+// Row-wise quantization (NVFP4 BS = 16 or MXFP4 BS = 32).
+// ---------------------------------------------------------------------------
+template <int BS, int RHT_N, bool SR>
+__global__ void __launch_bounds__(kThreads)
+quant_rows_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+                  uint32_t rht_mask, uint64_t sr_seed, uint32_t sr_stream,
+                  const float* __restrict__ amax_src, float* amax_out, float* s_dec_out,
+                  uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                  uint8_t* __restrict__ scales_mma, uint32_t* status) {
+  constexpr bool NV = (BS == 16);
+  constexpr int TPB = BS / 8;                 // threads per block
+  const int64_t cpr = cols >> 3, total = rows * cpr;
+  const int64_t S = cols / BS;
+  const int lane = threadIdx.x & 31;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+
+  float s_enc = 1.0f, s_dec = 1.0f;
+  if constexpr (NV) {
+    const float A = *amax_src;
+    if (!(A <= FLT_MAX)) {                    // Inf or NaN: precondition violated
+      if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, FP4_ERR_NONFINITE, 1);
+    }
+    nvfp4_global_scales(A, s_enc, s_dec);
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      if (amax_out != nullptr && amax_out != amax_src) *amax_out = A;
+    }
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0 && s_dec_out != nullptr) *s_dec_out = s_dec;
+
+  for (int64_t g0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x - lane); g0 < total;
+       g0 += stride) {
+    const int64_t g = g0 + lane;
+    const bool active = g < total;
+    const int64_t r = active ? g / cpr : 0, j = active ? g - r * cpr : 0;
+    float v[8];
+    if (active) {
+      bf16x8_to_f32(ld_nc_v4(x + r * ld + j * 8), v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+    }
+    if constexpr (RHT_N > 0) rht_chunk<RHT_N>(v, rht_mask, (int)(j % (RHT_N / 8)));
+
+    float bmax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
+#pragma unroll
+    for (int lx = 1; lx < TPB; lx <<= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xFFFFFFFFu, bmax, lx));
+
+    uint32_t sf;
+    float inv;
+    if constexpr (NV) {
+      const float t = __fdiv_rn(__fmul_rn(bmax, s_enc), 6.0f);
+      sf = e4m3_rn_sat(t);
+      inv = (sf == 0) ? 0.0f : __fdiv_rn(s_enc, e4m3_value(sf));
+    } else {
+      int e = (bmax == 0.0f) ? -127 : floor_log2_f32(bmax) - 2;
+      e = max(-127, min(127, e));
+      sf = (uint32_t)(e + 127);
+      inv = exp2_neg_exact(e);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], inv);
+
+    uint32_t packed;
+    if constexpr (!SR) {
+      packed = e2m1x8_rn(v);
+    } else {
+      const uint64_t i0 = (uint64_t)r * (uint64_t)cols + (uint64_t)(j * 8);
+      const U4 w0 = philox4x32_10(i0 >> 2, sr_stream, sr_seed);
+      const U4 w1 = philox4x32_10((i0 >> 2) + 1, sr_stream, sr_seed);
+      const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      packed = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) packed |= e2m1_sr(v[i], u[i]) << (4 * i);
+    }
+    if (active) {
+      *reinterpret_cast<uint32_t*>(codes + r * (cols >> 1) + j * 4) = packed;
+      if ((j % TPB) == 0) {
+        const int64_t s = j / TPB;
+        if (scales != nullptr) scales[r * S + s] = (uint8_t)sf;
+        if (scales_mma != nullptr) scales_mma[mma_sf_offset(r, s, (S + 3) & ~3LL)] = (uint8_t)sf;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Transposed quantization / amax: x [rows, cols] -> operand x^T [cols, rows],
+// blocks of BS run along x's rows.  64 x 64 tile per CTA (128 threads); the
+// thread owning (column k, half h) handles rows 32h .. 32h + 31 of the tile.
+// ---------------------------------------------------------------------------
+constexpr int kTile = 64;
+constexpr int kColThreads = 128;
+
+template <int BS, int RHT_N, bool SR, bool AMAX_ONLY>
+__global__ void __launch_bounds__(kColThreads)
+quant_cols_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+                  uint32_t rht_mask, uint64_t sr_seed, uint32_t sr_stream,
+                  const float* __restrict__ amax_src, float* amax_out, float* s_dec_out,
+                  uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                  uint8_t* __restrict__ scales_mma, uint32_t* status) {
+  constexpr bool NV = (BS == 16);
+  __shared__ __align__(16) __nv_bfloat16 tile[kTile][kTile];
+  __shared__ float red[kColThreads / 32];
+
+  const int64_t tiles_m = (rows + kTile - 1) / kTile, tiles_k = (cols + kTile - 1) / kTile;
+  const int64_t ntiles = tiles_m * tiles_k;
+  const int64_t S = rows / BS;             // blocks per row of x^T
+  const int t = threadIdx.x;
+  const int kk = t & 63, h = t >> 6;
+
+  float s_enc = 1.0f, s_dec = 1.0f;
+  if constexpr (NV && !AMAX_ONLY) {
+    const float A = *amax_src;
+    if (!(A <= FLT_MAX)) {
+      if (blockIdx.x == 0 && t == 0) set_status(status, FP4_ERR_NONFINITE, 2);
+    }
+    nvfp4_global_scales(A, s_enc, s_dec);
+    if (blockIdx.x == 0 && t == 0 && amax_out != nullptr && amax_out != amax_src) *amax_out = A;
+  }
+  if constexpr (!AMAX_ONLY) {
+    if (blockIdx.x == 0 && t == 0 && s_dec_out != nullptr) *s_dec_out = s_dec;
+  }
+  float m = 0.0f;
+
+  for (int64_t tile_id = blockIdx.x; tile_id < ntiles; tile_id += gridDim.x) {
+    const int64_t tm = tile_id / tiles_k, tk = tile_id - tm * tiles_k;
+    const int64_t m0 = tm * kTile, k0 = tk * kTile;
+    __syncthreads();                      // previous tile fully consumed
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int rr = (t >> 3) + 16 * it, cc = (t & 7) * 8;
+      uint4 u = make_uint4(0, 0, 0, 0);
+      if (m0 + rr < rows && k0 + cc < cols) u = ld_nc_v4(x + (m0 + rr) * ld + k0 + cc);
+      *reinterpret_cast<uint4*>(&tile[rr][cc]) = u;
+    }
+    __syncthreads();
+
+    const int64_t k = k0 + kk;
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __bfloat162float(tile[32 * h + i][kk]);
+
+    if constexpr (RHT_N > 0) {
+#pragma unroll
+      for (int base = 0; base < 32; base += RHT_N) {
+#pragma unroll
+        for (int i = 0; i < RHT_N; ++i)
+          if ((rht_mask >> i) & 1u) v[base + i] = -v[base + i];
+#pragma unroll
+        for (int hh = 1; hh < RHT_N; hh <<= 1) {
+#pragma unroll
+          for (int i = 0; i < RHT_N; ++i) {
+            if (i & hh) continue;
+            const float a = v[base + i], b = v[base + i + hh];
+            v[base + i] = __fadd_rn(a, b);
+            v[base + i + hh] = __fsub_rn(a, b);
+          }
+        }
+        const float c = rht_scale<RHT_N>();
+#pragma unroll
+        for (int i = 0; i < RHT_N; ++i) v[base + i] = __fmul_rn(v[base + i], c);
+      }
+    }
+
+    const int64_t mrow0 = m0 + 32 * h;    // first x row of this thread's run
+    if constexpr (AMAX_ONLY) {
+      if (k < cols) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (mrow0 + i < rows) m = absmax_keep_nan(m, v[i]);
+      }
+      continue;
+    } else {
+      if (k >= cols || mrow0 >= rows) continue;
+      uint32_t packed[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int b = 0; b < 32 / BS; ++b) {
+        if (mrow0 + b * BS >= rows) break;
+        float bmax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < BS; ++i) bmax = fmaxf(bmax, fabsf(v[b * BS + i]));
+        uint32_t sf;
+        float inv;
+        if constexpr (NV) {
+          const float tt = __fdiv_rn(__fmul_rn(bmax, s_enc), 6.0f);
+          sf = e4m3_rn_sat(tt);
+          inv = (sf == 0) ? 0.0f : __fdiv_rn(s_enc, e4m3_value(sf));
+        } else {
+          int e = (bmax == 0.0f) ? -127 : floor_log2_f32(bmax) - 2;
+          e = max(-127, min(127, e));
+          sf = (uint32_t)(e + 127);
+          inv = exp2_neg_exact(e);
+        }
+#pragma unroll
+        for (int i = 0; i < BS; ++i) v[b * BS + i] = __fmul_rn(v[b * BS + i], inv);
+        const int64_t s = (mrow0 + b * BS) / BS;
+        if (scales != nullptr) scales[k * S + s] = (uint8_t)sf;
+        if (scales_mma != nullptr) scales_mma[mma_sf_offset(k, s, (S + 3) & ~3LL)] = (uint8_t)sf;
+      }
+      if constexpr (!SR) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) packed[q] = e2m1x8_rn(&v[8 * q]);
+      } else {
+        const uint64_t i0 = (uint64_t)k * (uint64_t)rows + (uint64_t)mrow0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const U4 w = philox4x32_10((i0 >> 2) + q, sr_stream, sr_seed);
+          const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            packed[q >> 1] |= e2m1_sr(v[4 * q + i], u[i]) << (4 * ((4 * q + i) & 7));
+        }
+      }
+      uint8_t* dst = codes + k * (rows >> 1) + (mrow0 >> 1);
+      *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+      if (mrow0 + 16 < rows) *reinterpret_cast<uint2*>(dst + 8) = make_uint2(packed[2], packed[3]);
+    }
+  }
+  if constexpr (AMAX_ONLY) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if ((t & 31) == 0) red[t >> 5] = m;
+    __syncthreads();
+    if (t == 0) {
+      float mm = red[0];
+      for (int w = 1; w < kColThreads / 32; ++w) mm = fmaxf(mm, red[w]);
+      atomicMax(reinterpret_cast<unsigned int*>(amax_out), __float_as_uint(mm));
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// NVFP4 16x16 2-D quantization (round to nearest): one E4M3 scale per tile.
+// 64 x 64 region per CTA, 256 threads.  Emits W and W^T from the same codes.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+quant_2d_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+                const float* __restrict__ amax_src, float* s_dec_out, float* s_dec_out_t,
+                float* amax_out, float* amax_out_t, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                uint8_t* __restrict__ scales_mma, uint8_t* __restrict__ codes_t,
+                uint8_t* __restrict__ scales_t, uint8_t* __restrict__ scales_mma_t,
+                uint32_t* status) {
+  __shared__ float tile[kTile][kTile + 1];
+  __shared__ float tinv[16];
+  __shared__ uint32_t tsf[16];
+  const int t = threadIdx.x;
+  const int64_t tiles_r = (rows + kTile - 1) / kTile, tiles_c = (cols + kTile - 1) / kTile;
+  const int64_t S = cols / 16, St = rows / 16;
+
+  const float A = *amax_src;
+  if (!(A <= FLT_MAX) && blockIdx.x == 0 && t == 0) set_status(status, FP4_ERR_NONFINITE, 3);
+  float s_enc, s_dec;
+  nvfp4_global_scales(A, s_enc, s_dec);
+  if (blockIdx.x == 0 && t == 0) {
+    if (s_dec_out) *s_dec_out = s_dec;
+    if (s_dec_out_t) *s_dec_out_t = s_dec;
+    if (amax_out && amax_out != amax_src) *amax_out = A;
+    if (amax_out_t && amax_out_t != amax_src) *amax_out_t = A;
+  }
+
+  for (int64_t tid = blockIdx.x; tid < tiles_r * tiles_c; tid += gridDim.x) {
+    const int64_t r0 = (tid / tiles_c) * kTile, c0 = (tid % tiles_c) * kTile;
+    __syncthreads();
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+      const int rr = (t >> 3) + 32 * it, cc = (t & 7) * 8;
+      float v[8];
+      if (r0 + rr < rows && c0 + cc < cols) {
+        bf16x8_to_f32(ld_nc_v4(x + (r0 + rr) * ld + c0 + cc), v);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) tile[rr][cc + i] = v[i];
+    }
+    __syncthreads();
+    {  // tile max: 16 threads per 16x16 tile, one tile row each
+      const int q = t >> 4, rr = t & 15;
+      const int tr = q >> 2, tc = q & 3;
+      float bm = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) bm = fmaxf(bm, fabsf(tile[tr * 16 + rr][tc * 16 + i]));
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xFFFFFFFFu, bm, o));
+      if (rr == 0) {
+        const float tt = __fdiv_rn(__fmul_rn(bm, s_enc), 6.0f);
+        const uint32_t sf = e4m3_rn_sat(tt);
+        tsf[q] = sf;
+        tinv[q] = (sf == 0) ? 0.0f : __fdiv_rn(s_enc, e4m3_value(sf));
+        const int64_t gr = r0 / 16 + tr, gc = c0 / 16 + tc;
+        if (gr < St && gc < S) {
+          if (scales) scales[gr * S + gc] = (uint8_t)sf;
+          if (scales_t) scales_t[gc * St + gr] = (uint8_t)sf;
+        }
+      }
+    }
+    __syncthreads();
+    {  // W: row r0 + (t >> 2), 16-block (t & 3)
+      const int rr = t >> 2, kb = t & 3;
+      const int64_t r = r0 + rr, c = c0 + kb * 16;
+      if (r < rows && c < cols) {
+        const int q = (rr >> 4) * 4 + kb;
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(tile[rr][kb * 16 + i], tinv[q]);
+        if (codes) {
+          *reinterpret_cast<uint2*>(codes + r * (cols >> 1) + (c >> 1)) =
+              make_uint2(e2m1x8_rn(v), e2m1x8_rn(v + 8));
+        }
+        if (scales_mma) scales_mma[mma_sf_offset(r, c / 16, (S + 3) & ~3LL)] = (uint8_t)tsf[q];
+      }
+    }
+    {  // W^T: row c0 + (t >> 2) of W^T (a column of W), 16-block (t & 3) of W rows
+      const int cc = t >> 2, rb = t & 3;
+      const int64_t k = c0 + cc, r = r0 + rb * 16;
+      if (k < cols && r < rows) {
+        const int q = rb * 4 + (cc >> 4);
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(tile[rb * 16 + i][cc], tinv[q]);
+        if (codes_t) {
+          *reinterpret_cast<uint2*>(codes_t + k * (rows >> 1) + (r >> 1)) =
+              make_uint2(e2m1x8_rn(v), e2m1x8_rn(v + 8));
+        }
+        if (scales_mma_t) scales_mma_t[mma_sf_offset(k, r / 16, (St + 3) & ~3LL)] = (uint8_t)tsf[q];
+      }
+    }
+  }
+}
+
+int grid_for(int64_t work_items, int per_block, int max_blocks_per_sm) {
+  int64_t need = (work_items + per_block - 1) / per_block;
+  const int64_t cap = (int64_t)sm_count() * max_blocks_per_sm;
+  if (need > cap) need = cap;
+  if (need < 1) need = 1;
+  return (int)need;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// Launchers
+// ---------------------------------------------------------------------------
+cudaError_t launch_amax_rows(const void* x, int64_t rows, int64_t cols, int64_t ld, int rht_n,
+                             uint32_t mask, float* amax, cudaStream_t s) {
+  const int grid = grid_for(rows * (cols / 8), kThreads, 8);
+  auto xp = static_cast<const __nv_bfloat16*>(x);
+  if (rht_n == 16) amax_rows_kernel<16><<<grid, kThreads, 0, s>>>(xp, rows, cols, ld, mask, amax);
+  else if (rht_n == 32) amax_rows_kernel<32><<<grid, kThreads, 0, s>>>(xp, rows, cols, ld, mask, amax);
+  else amax_rows_kernel<0><<<grid, kThreads, 0, s>>>(xp, rows, cols, ld, mask, amax);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_amax_cols(const void* x, int64_t rows, int64_t cols, int64_t ld, int rht_n,
+                             uint32_t mask, float* amax, cudaStream_t s) {
+  const int64_t ntiles = ((rows + kTile - 1) / kTile) * ((cols + kTile - 1) / kTile);
+  const int grid = grid_for(ntiles, 1, 16);
+  auto xp = static_cast<const __nv_bfloat16*>(x);
+#define FP4_AMAXC(N) quant_cols_kernel<16, N, false, true><<<grid, kColThreads, 0, s>>>( \
+      xp, rows, cols, ld, mask, 0, 0, nullptr, amax, nullptr, nullptr, nullptr, nullptr, nullptr)
+  if (rht_n == 16) FP4_AMAXC(16);
+  else if (rht_n == 32) FP4_AMAXC(32);
+  else FP4_AMAXC(0);
+#undef FP4_AMAXC
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+template <int BS, int RHT_N, bool SR>
+static void rows_variant(const RowQuantArgs& a, int grid, cudaStream_t s) {
+  quant_rows_kernel<BS, RHT_N, SR><<<grid, kThreads, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(a.x), a.rows, a.cols, a.ld, a.rht_mask, a.sr_seed,
+      a.sr_stream, a.amax_src, a.amax_out, a.s_dec, a.codes, a.scales, a.scales_mma, a.status);
+}
+
+template <int BS, int RHT_N, bool SR>
+static void cols_variant(const RowQuantArgs& a, int grid, cudaStream_t s) {
+  quant_cols_kernel<BS, RHT_N, SR, false><<<grid, kColThreads, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(a.x), a.rows, a.cols, a.ld, a.rht_mask, a.sr_seed,
+      a.sr_stream, a.amax_src, a.amax_out, a.s_dec, a.codes, a.scales, a.scales_mma, a.status);
+}
+
+#define FP4_DISPATCH(FN, a, grid, s)                                                    \
+  do {                                                                                  \
+    const bool sr = (a).round == FP4_SR;                                                \
+    if ((a).fmt == FP4_NVFP4) {                                                         \
+      if ((a).rht_n == 16) { sr ? FN<16, 16, true>(a, grid, s) : FN<16, 16, false>(a, grid, s); } \
+      else if ((a).rht_n == 32) { sr ? FN<16, 32, true>(a, grid, s) : FN<16, 32, false>(a, grid, s); } \
+      else { sr ? FN<16, 0, true>(a, grid, s) : FN<16, 0, false>(a, grid, s); }          \
+    } else {                                                                            \
+      if ((a).rht_n == 16) { sr ? FN<32, 16, true>(a, grid, s) : FN<32, 16, false>(a, grid, s); } \
+      else if ((a).rht_n == 32) { sr ? FN<32, 32, true>(a, grid, s) : FN<32, 32, false>(a, grid, s); } \
+      else { sr ? FN<32, 0, true>(a, grid, s) : FN<32, 0, false>(a, grid, s); }          \
+    }                                                                                   \
+  } while (0)
+
+cudaError_t launch_quant_rows(const RowQuantArgs& a, cudaStream_t s) {
+  const int grid = grid_for(a.rows * (a.cols / 8), kThreads, 8);
+  FP4_DISPATCH(rows_variant, a, grid, s);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_cols(const RowQuantArgs& a, cudaStream_t s) {
+  const int64_t ntiles = ((a.rows + kTile - 1) / kTile) * ((a.cols + kTile - 1) / kTile);
+  const int grid = grid_for(ntiles, 1, 16);
+  FP4_DISPATCH(cols_variant, a, grid, s);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_2d(const Quant2DArgs& a, cudaStream_t s) {
+  const int64_t ntiles = ((a.rows + kTile - 1) / kTile) * ((a.cols + kTile - 1) / kTile);
+  const int grid = grid_for(ntiles, 1, 8);
+  quant_2d_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(a.x), a.rows, a.cols,
+                                       a.ld, a.amax_src, a.s_dec, a.s_dec_t, a.amax_out,
+                                       a.amax_out_t, a.codes,
+                                       a.scales, a.scales_mma, a.codes_t, a.scales_t,
+                                       a.scales_mma_t, a.status);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace fp4impl

@@ -1,0 +1,242 @@
+/*
+ * fp4.h -- C ABI of libfp4fqt.so, a B200 (sm_100a) library for the
+ * fully-quantized FP4 linear layer: block quantization of BF16 tensors to
+ * NVFP4 / MXFP4 and the three block-scaled FP4 GEMMs of a linear layer
+ * (fprop, dgrad, wgrad), accumulated in FP32 on the tensor cores.
+ *
+ * What is computed (page title, section):
+ *   - "FP4" (Robots Atlas), How it works: values are cast to 4-bit E2M1;
+ *     a tensor is split into small blocks (16 values for NVFP4, 32 for
+ *     MXFP4), each with its own scale (E4M3 for NVFP4, E8M0 for MXFP4);
+ *     NVFP4 adds one FP32 scale for the whole tensor; matrix products run
+ *     on the tensor cores in FP4 and accumulate in higher precision; random
+ *     Hadamard transforms, two-dimensional quantization and stochastic
+ *     rounding of gradients stabilise training.
+ *   - "FP4" (Robots Atlas), Components: the E2M1 levels 0, 0.5, 1, 1.5, 2,
+ *     3, 4, 6 and their negatives; NVFP4 and MXFP4 block formats.
+ *   - "FP4 All the Way: Fully Quantized Training of LLMs", Key points:
+ *     NVFP4, round-to-nearest in the forward pass, stochastic rounding in
+ *     the backward and update passes.
+ *   - "Quartet: Native FP4 Training Can Be Optimal for Large Language
+ *     Models", Approach: all three linear-layer GEMMs in FP4, round-to-
+ *     nearest backward with block-wise Hadamard rotations (the MXFP4 mode).
+ *
+ * Conventions shared by every entry point:
+ *   - Every tensor pointer is DEVICE memory owned by the caller.  The
+ *     library allocates no device memory and keeps no global mutable state;
+ *     calls on different streams do not interfere unless they share
+ *     buffers.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  All work is enqueued asynchronously on it; no entry point
+ *     synchronises except fp4_read_device_status.
+ *   - Argument errors are returned synchronously, before anything is
+ *     enqueued.  A failed launch returns FP4_ERR_CUDA.  Conditions found on
+ *     the device (non-finite amax, expired bounded wait) are OR-ed into the
+ *     status word at the start of the workspace `ws`, read with
+ *     fp4_read_device_status; they are sticky until fp4_clear_device_status.
+ *   - Matrices are row-major.  Packed FP4 codes: two per byte, element 2j in
+ *     the low nibble of byte j.  A code is sign (bit 3), exponent (bits 2-1),
+ *     mantissa (bit 0).  Pointers must be 16-byte aligned.
+ *   - Stochastic-rounding draws are counter-based: element i (row-major
+ *     index in the quantized operand's own logical layout) uses word i mod 4
+ *     of Philox4x32-10 with key (seed lo, seed hi) and counter
+ *     (i/4 lo, i/4 hi, stream, 0), so results do not depend on the launch
+ *     configuration.  The Hadamard sign vector d (d_j = -1 iff bit 31 of
+ *     draw j of stream 0x48414441 under the RHT seed) is shared by every
+ *     block of both operands of a GEMM.
+ */
+#ifndef FP4FQT_FP4_H
+#define FP4FQT_FP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FP4_ABI_VERSION 1
+
+/* ---------------------------------------------------------------------- */
+/* Status codes                                                            */
+/* ---------------------------------------------------------------------- */
+typedef enum fp4_status {
+  FP4_OK = 0,
+  FP4_ERR_NULL = 1,        /* a required pointer is NULL                        */
+  FP4_ERR_SHAPE = 2,       /* sizes violate the divisibility rules              */
+  FP4_ERR_ALIGN = 3,       /* a pointer or leading dimension is not aligned     */
+  FP4_ERR_FORMAT = 4,      /* inconsistent format / block / rounding request    */
+  FP4_ERR_WORKSPACE = 5,   /* workspace missing or smaller than required        */
+  FP4_ERR_CUDA = 6,        /* a CUDA call or kernel launch failed               */
+  FP4_ERR_NONFINITE = 7,   /* device: a tensor amax was Inf or NaN              */
+  FP4_ERR_TIMEOUT = 8,     /* device: a bounded wait inside a GEMM expired      */
+  FP4_ERR_UNSUPPORTED = 9  /* a valid request this build does not implement     */
+} fp4_status;
+
+/* Values of the int32_t selector fields below. */
+enum { FP4_NVFP4 = 0, FP4_MXFP4 = 1 };            /* format                  */
+enum { FP4_RTN = 0, FP4_SR = 1 };                 /* rounding                */
+enum { FP4_BLOCK_1D = 0, FP4_BLOCK_2D = 1 };      /* 1x16 / 1x32, or 16x16    */
+enum { FP4_OUT_BF16 = 0, FP4_OUT_F32 = 1 };       /* GEMM output type         */
+enum { FQT_RHT_FPROP = 1, FQT_RHT_DGRAD = 2, FQT_RHT_WGRAD = 4 };
+
+/* ---------------------------------------------------------------------- */
+/* A quantized operand (all buffers caller-allocated device memory).       */
+/*                                                                         */
+/* codes      [rows, cols/2] bytes.                                        */
+/* scales     logical block scales, may be NULL:                           */
+/*              NVFP4 1-D: [rows, cols/16] E4M3; NVFP4 2-D: [rows/16,      */
+/*              cols/16] E4M3 (one per 16x16 tile); MXFP4: [rows, cols/32]  */
+/*              E8M0.                                                       */
+/* scales_mma the same scales in the tensor-core layout, may be NULL;      */
+/*              required by fp4_gemm.  One byte per (row, block of 16 or 32 */
+/*              columns), 2-D tile scales replicated to each of the tile's  */
+/*              16 rows, arranged in 512-byte atoms of 128 rows x 4 blocks: */
+/*              byte offset of (r, s) with S = cols/blocksize blocks a row: */
+/*                ((r/128) * (S/4) + s/4) * 512                             */
+/*                  + (r%32)*16 + ((r%128)/32)*4 + s%4.                     */
+/*              Needs rows % 128 == 0 and S % 4 == 0; size rows*S bytes.    */
+/* amax       [1] float: tensor amax (of the rotated values when a Hadamard */
+/*              transform is applied); written by fp4_quantize.  NVFP4 only */
+/*              (may be NULL for MXFP4).                                    */
+/* s_dec      [1] float: per-tensor decode scale.  NVFP4: amax/2688 (1 when */
+/*              amax = 0); MXFP4: 1.  Written by fp4_quantize.              */
+/* ---------------------------------------------------------------------- */
+typedef struct fp4_qtensor {
+  uint8_t* codes;
+  uint8_t* scales;
+  uint8_t* scales_mma;
+  float* amax;
+  float* s_dec;
+  int64_t rows;
+  int64_t cols;
+  int32_t fmt;      /* FP4_NVFP4 / FP4_MXFP4 */
+  int32_t block;    /* FP4_BLOCK_1D / FP4_BLOCK_2D */
+} fp4_qtensor;
+
+/* Byte sizes of the buffers of a quantized operand of logical shape
+ * [rows, cols]; any output pointer may be NULL. */
+void fp4_qtensor_sizes(int64_t rows, int64_t cols, int32_t fmt, int32_t block,
+                       size_t* codes_bytes, size_t* scales_bytes, size_t* scales_mma_bytes);
+
+/* ---------------------------------------------------------------------- */
+/* Quantization request.                                                   */
+/* The row-wise output quantizes x along its columns (blocks run along a   */
+/* row); the transposed output quantizes x^T, i.e. blocks run down x's      */
+/* columns, and is stored as a [cols, rows] operand.                        */
+/* ---------------------------------------------------------------------- */
+typedef struct fp4_qparams {
+  int32_t fmt;            /* FP4_NVFP4 or FP4_MXFP4                                  */
+  int32_t block;          /* FP4_BLOCK_1D, or FP4_BLOCK_2D (NVFP4 weights, RTN only) */
+  int32_t round;          /* rounding of the row-wise output                         */
+  int32_t round_t;        /* rounding of the transposed output                       */
+  int32_t rht_n;          /* 0, 16 or 32: Hadamard block of the row-wise output      */
+  int32_t rht_n_t;        /* 0, 16 or 32: Hadamard block of the transposed output    */
+  uint64_t rht_seed;      /* seed of the Hadamard sign vector                        */
+  uint64_t sr_seed;       /* seed of the stochastic-rounding draws                   */
+  uint32_t sr_stream;     /* Philox stream of the row-wise output                    */
+  uint32_t sr_stream_t;   /* Philox stream of the transposed output                  */
+  const float* amax_in;   /* optional device float: use this amax for the row-wise  */
+                          /* output instead of computing it (single-pass encode)     */
+  const float* amax_in_t; /* same for the transposed output                          */
+} fp4_qparams;
+
+/* Defaults: NVFP4 1-D, RTN, no Hadamard, seed 0, streams 0. */
+void fp4_qparams_default(fp4_qparams* p);
+
+/* Workspace bytes needed by fp4_gemm for an M x N x K product (also enough
+ * for every other entry point).  At least 256: the status block. */
+size_t fp4_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/* Quantize x (BF16, [rows, cols] with leading dimension ld >= cols, in
+ * elements, ld % 8 == 0) into `out` (row-wise, may be NULL) and/or `out_t`
+ * (transposed, may be NULL).  Shape rules: NVFP4 1-D needs cols % 16 == 0
+ * for `out` and rows % 16 == 0 for `out_t`; MXFP4 the same with 32; NVFP4
+ * 2-D needs rows % 16 == 0 and cols % 16 == 0 and produces W (`out`) and
+ * W^T (`out_t`) from one tile scale per 16x16 tile (identical codes,
+ * transposed).  A Hadamard block must divide the blocked dimension.  The
+ * qtensors' rows/cols/fmt/block must describe the requested outputs.
+ * `ws` may be NULL (device conditions are then not recorded).
+ * Two passes over x (amax, then encode) unless the amax is supplied. */
+fp4_status fp4_quantize(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                        const fp4_qparams* params, fp4_qtensor* out, fp4_qtensor* out_t,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/* Block-scaled FP4 GEMM, both operands K-major ("NT"):
+ *   C[m, n] = alpha * s_dec(a) * s_dec(b) * sum_k a_hat[m, k] * b_hat[n, k]
+ * with a_hat = e2m1(code) * block scale, M = a->rows, N = b->rows,
+ * K = a->cols = b->cols, accumulated in FP32 on the tensor cores.
+ * Requires a->fmt == b->fmt, both scales_mma set, M % 128 == 0,
+ * N % 128 == 0, K % 64 == 0, K > 0.  C is [M, ldc] of `out_dtype` with
+ * ldc >= N and ldc * element size a multiple of 16 bytes.
+ * c_amax (nullable device float) receives max |C| over the output.
+ * ws must hold fp4_workspace_bytes(M, N, K) bytes. */
+fp4_status fp4_gemm(const fp4_qtensor* a, const fp4_qtensor* b, float alpha, void* c,
+                    int64_t ldc, int32_t out_dtype, float* c_amax, void* ws,
+                    size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Linear layer  Y = X W^T  with X [M, K], W [N, K], dY [M, N]:            */
+/*   fprop  Y  = X . W^T      (contract K)                                 */
+/*   dgrad  dX = dY . W       (contract N; uses W^T stored [K, N])          */
+/*   wgrad  dW = dY^T . X     (contract M; uses dY^T [N, M] and X^T [K, M]) */
+/* ---------------------------------------------------------------------- */
+typedef struct fqt_linear_cfg {
+  int32_t fmt;        /* FP4_NVFP4 or FP4_MXFP4                                   */
+  int32_t w_block;    /* NVFP4: FP4_BLOCK_2D (16x16 weight tiles) or FP4_BLOCK_1D  */
+  int32_t round_fwd;  /* rounding of X and W for fprop                            */
+  int32_t round_bwd;  /* rounding of dY (dgrad and wgrad operands)                */
+  int32_t round_x_t;  /* rounding of X^T, the wgrad ("update pass") operand       */
+  int32_t rht_mask;   /* FQT_RHT_* bits: GEMMs whose operands are rotated first    */
+  int32_t rht_n;      /* Hadamard block: 16 (NVFP4 default) or 32 (MXFP4 default)  */
+  int32_t out_dtype;  /* FP4_OUT_BF16 / FP4_OUT_F32 for Y and dX (dW is FP32)      */
+  uint64_t seed;      /* stochastic-rounding and Hadamard seed                    */
+} fqt_linear_cfg;
+
+/* Defaults. NVFP4: 2-D weights, RTN forward, SR for dY and X^T, no Hadamard.
+ * MXFP4: 1-D weights, RTN everywhere, 32-point Hadamard on all three GEMMs.
+ * Philox streams used by the layer: dY row-wise 1, dY^T 2, X^T 3. */
+void fqt_linear_cfg_default(fqt_linear_cfg* cfg, int32_t fmt);
+
+/* Quantized operands of one layer (caller-allocated, shapes as listed). */
+typedef struct fqt_saved {
+  fp4_qtensor xq;     /* X   [M, K]  fprop A   */
+  fp4_qtensor xq_t;   /* X^T [K, M]  wgrad B   */
+  fp4_qtensor wq;     /* W   [N, K]  fprop B   */
+  fp4_qtensor wq_t;   /* W^T [K, N]  dgrad B   */
+  fp4_qtensor dyq;    /* dY  [M, N]  dgrad A   */
+  fp4_qtensor dyq_t;  /* dY^T [N, M] wgrad A   */
+} fqt_saved;
+
+/* Forward: quantize X (row-wise and transposed) and W (both orientations),
+ * then Y = fprop.  x, w BF16; y of cfg->out_dtype, [M, N] dense. */
+fp4_status fqt_linear_fwd(const fqt_linear_cfg* cfg, int64_t M, int64_t N, int64_t K,
+                          const void* x, const void* w, void* y, fqt_saved* saved,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* Backward: quantize dY (row-wise and transposed), then dX = dgrad
+ * ([M, K], cfg->out_dtype) and dW = wgrad ([N, K], FP32). */
+fp4_status fqt_linear_bwd(const fqt_linear_cfg* cfg, int64_t M, int64_t N, int64_t K,
+                          const void* dy, fqt_saved* saved, void* dx, float* dw,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, then return the device status word of `ws`
+ * (FP4_OK when no device condition was recorded). */
+fp4_status fp4_read_device_status(const void* ws, void* stream);
+
+/* Enqueue a reset of the device status word of `ws`. */
+fp4_status fp4_clear_device_status(void* ws, void* stream);
+
+const char* fp4_status_str(int32_t status);
+int32_t fp4_abi_version(void);
+
+/* Number of CUDA kernels this library has enqueued in the calling process
+ * since it was loaded (all devices, all streams).  Host-side counter, no
+ * synchronisation; used to attribute work in a timed region. */
+uint64_t fp4_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP4FQT_FP4_H */

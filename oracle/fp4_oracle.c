@@ -386,6 +386,47 @@ int orc_nvfp4_quantize_1d(const float* x, int64_t R, int64_t C, int64_t row_offs
  * [FP4] How it works: "two-dimensional quantization" as a stabiliser; the
  * 16x16 tile is the 2-D analogue of the 16-value block.  One E4M3 scale per
  * 16x16 tile, scales laid out [R/16, C/16]; codes [R, C/2] as in 1-D. */
+typedef struct {
+  const float* x;
+  int64_t R, C;
+  float s_enc;
+  uint8_t* codes;
+  uint8_t* scales;
+} q2d_ctx;
+
+/* Tile rows [t0, t1) of the 16x16 grid. */
+static void nvfp4_2d_worker(void* p, int64_t t0, int64_t t1) {
+  q2d_ctx* q = (q2d_ctx*)p;
+  const int64_t C = q->C, tc = C / 16;
+  for (int64_t i = t0; i < t1; ++i) {
+    for (int64_t j = 0; j < tc; ++j) {
+      float bmax = 0.0f;
+      for (int a = 0; a < 16; ++a)
+        for (int b = 0; b < 16; ++b) {
+          float v = fabsf(q->x[(i * 16 + a) * C + j * 16 + b]);
+          if (v > bmax) bmax = v;
+        }
+      float t = (bmax * q->s_enc) / 6.0f;
+      uint8_t sf = orc_e4m3_rne_sat(t);
+      float sfv = (float)orc_e4m3_value(sf);
+      float inv = (sf == 0) ? 0.0f : q->s_enc / sfv;
+      q->scales[i * tc + j] = sf;
+      for (int a = 0; a < 16; ++a)
+        for (int b = 0; b < 16; ++b) {
+          int64_t r = i * 16 + a, c = j * 16 + b;
+          uint8_t code = orc_e2m1_rtn(q->x[r * C + c] * inv);
+          uint8_t* byte = &q->codes[r * (C / 2) + c / 2];
+          if ((c & 1) == 0) *byte = (uint8_t)((*byte & 0xF0) | code);
+          else *byte = (uint8_t)((*byte & 0x0F) | (code << 4));
+        }
+    }
+  }
+}
+
+/* NVFP4 16x16 2-D quantization (weights, round to nearest).
+ * [FP4] How it works: "two-dimensional quantization" as a stabiliser; the
+ * 16x16 tile is the 2-D analogue of the 16-value block.  One E4M3 scale per
+ * 16x16 tile, scales laid out [R/16, C/16]; codes [R, C/2] as in 1-D. */
 int orc_nvfp4_quantize_2d(const float* x, int64_t R, int64_t C, const float* amax_in,
                           uint8_t* codes, uint8_t* scales, float* amax_out,
                           float* s_dec_out) {
@@ -394,30 +435,8 @@ int orc_nvfp4_quantize_2d(const float* x, int64_t R, int64_t C, const float* ama
   float s_enc, s_dec;
   orc_nvfp4_global_scales(A, &s_enc, &s_dec);
   memset(codes, 0, (size_t)(R * C / 2));
-  const int64_t tr = R / 16, tc = C / 16;
-  for (int64_t i = 0; i < tr; ++i) {
-    for (int64_t j = 0; j < tc; ++j) {
-      float bmax = 0.0f;
-      for (int a = 0; a < 16; ++a)
-        for (int b = 0; b < 16; ++b) {
-          float v = fabsf(x[(i * 16 + a) * C + j * 16 + b]);
-          if (v > bmax) bmax = v;
-        }
-      float t = (bmax * s_enc) / 6.0f;
-      uint8_t sf = orc_e4m3_rne_sat(t);
-      float sfv = (float)orc_e4m3_value(sf);
-      float inv = (sf == 0) ? 0.0f : s_enc / sfv;
-      scales[i * tc + j] = sf;
-      for (int a = 0; a < 16; ++a)
-        for (int b = 0; b < 16; ++b) {
-          int64_t r = i * 16 + a, c = j * 16 + b;
-          uint8_t code = orc_e2m1_rtn(x[r * C + c] * inv);
-          uint8_t* byte = &codes[r * (C / 2) + c / 2];
-          if ((c & 1) == 0) *byte = (uint8_t)((*byte & 0xF0) | code);
-          else *byte = (uint8_t)((*byte & 0x0F) | (code << 4));
-        }
-    }
-  }
+  q2d_ctx q = {x, R, C, s_enc, codes, scales};
+  parallel_rows(nvfp4_2d_worker, &q, R / 16);
   if (amax_out) *amax_out = A;
   if (s_dec_out) *s_dec_out = s_dec;
   return 0;

@@ -1,0 +1,95 @@
+"""The C-ABI library loads on a machine without a GPU, exports every symbol
+include/fp4.h declares, and rejects bad arguments before touching CUDA."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import fp4_fully_quantized_b200 as F
+from conftest import ROOT
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "fp4.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(", src)
+    keep = [n for n in names if n.startswith(("fp4_", "fqt_"))]
+    return sorted(set(keep))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from fp4_fully_quantized_b200 import build
+    build.build()
+    return F.load()
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared_functions()
+    assert set(declared) == set(F.EXPORTS), (declared, F.EXPORTS)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_host_only_helpers(lib):
+    assert lib.fp4_abi_version() == 1
+    assert lib.fp4_status_str(7) == b"a tensor amax was Inf or NaN"
+    assert F.qtensor_sizes(256, 512, F.NVFP4, F.BLOCK_1D) == (256 * 256, 256 * 32, 256 * 32)
+    assert F.qtensor_sizes(256, 512, F.NVFP4, F.BLOCK_2D)[1] == 16 * 32
+    assert F.qtensor_sizes(128, 96, F.MXFP4, F.BLOCK_1D) == (128 * 48, 128 * 3, 128 * 4)
+    assert F.qtensor_sizes(100, 64, F.NVFP4, F.BLOCK_1D)[2] == 128 * 4
+    assert lib.fp4_workspace_bytes(128, 128, 64) >= 256
+    nv = F.linear_cfg(F.NVFP4)
+    assert (nv.w_block, nv.round_fwd, nv.round_bwd, nv.round_x_t, nv.rht_mask) == (
+        F.BLOCK_2D, F.RTN, F.SR, F.SR, 0)
+    mx = F.linear_cfg(F.MXFP4)
+    assert (mx.w_block, mx.round_bwd, mx.rht_mask, mx.rht_n) == (F.BLOCK_1D, F.RTN, 7, 32)
+
+
+def _q(rows, cols, fmt=0, block=0):
+    return F.QTensorC(C.c_void_p(4096), C.c_void_p(4096), C.c_void_p(4096), C.c_void_p(4096),
+                      C.c_void_p(4100), rows, cols, fmt, block)
+
+
+def test_argument_errors_return_before_launch(lib):
+    p = F.QParamsC()
+    lib.fp4_qparams_default(C.byref(p))
+    q = _q(32, 64)
+    fake_x = C.c_void_p(1 << 20)
+    # no output at all
+    assert lib.fp4_quantize(fake_x, 32, 64, 64, C.byref(p), None, None, None, 0, None) == 1
+    # misaligned input / leading dimension
+    assert lib.fp4_quantize(C.c_void_p((1 << 20) + 2), 32, 64, 64, C.byref(p), C.byref(q), None,
+                            None, 0, None) == 3
+    assert lib.fp4_quantize(fake_x, 32, 64, 66, C.byref(p), C.byref(q), None, None, 0, None) == 3
+    # cols not a multiple of 16
+    q2 = _q(32, 40)
+    assert lib.fp4_quantize(fake_x, 32, 40, 40, C.byref(p), C.byref(q2), None, None, 0, None) == 2
+    # qtensor shape disagrees with the request
+    assert lib.fp4_quantize(fake_x, 32, 128, 128, C.byref(p), C.byref(q), None, None, 0, None) == 2
+    # 2-D blocks are NVFP4 only; bad Hadamard size; bad rounding
+    p2 = F.QParamsC(); lib.fp4_qparams_default(C.byref(p2)); p2.fmt = 1; p2.block = 1
+    assert lib.fp4_quantize(fake_x, 32, 64, 64, C.byref(p2), C.byref(q), None, None, 0, None) == 4
+    p3 = F.QParamsC(); lib.fp4_qparams_default(C.byref(p3)); p3.rht_n = 8
+    assert lib.fp4_quantize(fake_x, 32, 64, 64, C.byref(p3), C.byref(q), None, None, 0, None) == 4
+    p4 = F.QParamsC(); lib.fp4_qparams_default(C.byref(p4)); p4.round = 5
+    assert lib.fp4_quantize(fake_x, 32, 64, 64, C.byref(p4), C.byref(q), None, None, 0, None) == 4
+    # workspace too small
+    assert lib.fp4_quantize(fake_x, 32, 64, 64, C.byref(p), C.byref(q), None, C.c_void_p(4096), 8,
+                            None) == 5
+    # GEMM: shape rules (M, N multiples of 128; K multiple of 64), formats, workspace
+    a, b = _q(128, 128), _q(256, 128)
+    ws = C.c_void_p(1 << 21)
+    c = C.c_void_p(1 << 22)
+    assert lib.fp4_gemm(C.byref(_q(96, 128)), C.byref(b), 1.0, c, 256, 1, None, ws, 256, None) == 2
+    assert lib.fp4_gemm(C.byref(a), C.byref(_q(256, 96)), 1.0, c, 256, 1, None, ws, 256, None) == 2
+    assert lib.fp4_gemm(C.byref(a), C.byref(_q(256, 128, 1)), 1.0, c, 256, 1, None, ws, 256,
+                        None) == 4
+    assert lib.fp4_gemm(C.byref(a), C.byref(b), 1.0, c, 200, 1, None, ws, 256, None) == 3
+    assert lib.fp4_gemm(C.byref(a), C.byref(b), 1.0, c, 256, 1, None, None, 0, None) == 5
+    assert lib.fp4_gemm(C.byref(a), C.byref(b), 1.0, c, 256, 7, None, ws, 256, None) == 4
+    # linear layer: 2-D weights cannot take a rotation on fprop/dgrad
+    cfg = F.linear_cfg(F.NVFP4, rht_mask=F.RHT_FPROP)
+    assert lib.fqt_linear_fwd(C.byref(cfg), 128, 128, 128, fake_x, fake_x, fake_x,
+                              C.byref(F.SavedC()), ws, 256, None) == 9
