@@ -160,7 +160,7 @@ quant_rows_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t col
     if constexpr (NV) {
       const float t = __fdiv_rn(__fmul_rn(bmax, s_enc), 6.0f);
       sf = e4m3_rn_sat(t);
-      inv = (sf == 0) ? 0.0f : __fdiv_rn(s_enc, e4m3_value(sf));
+      inv = (sf == 0) ? 0.0f : fminf(__fdiv_rn(s_enc, e4m3_value(sf)), FLT_MAX);
     } else {
       int e = (bmax == 0.0f) ? -127 : floor_log2_f32(bmax) - 2;
       e = max(-127, min(127, e));
@@ -294,7 +294,7 @@ quant_cols_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t col
         if constexpr (NV) {
           const float tt = __fdiv_rn(__fmul_rn(bmax, s_enc), 6.0f);
           sf = e4m3_rn_sat(tt);
-          inv = (sf == 0) ? 0.0f : __fdiv_rn(s_enc, e4m3_value(sf));
+          inv = (sf == 0) ? 0.0f : fminf(__fdiv_rn(s_enc, e4m3_value(sf)), FLT_MAX);
         } else {
           int e = (bmax == 0.0f) ? -127 : floor_log2_f32(bmax) - 2;
           e = max(-127, min(127, e));
@@ -397,7 +397,7 @@ quant_2d_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols,
         const float tt = __fdiv_rn(__fmul_rn(bm, s_enc), 6.0f);
         const uint32_t sf = e4m3_rn_sat(tt);
         tsf[q] = sf;
-        tinv[q] = (sf == 0) ? 0.0f : __fdiv_rn(s_enc, e4m3_value(sf));
+        tinv[q] = (sf == 0) ? 0.0f : fminf(__fdiv_rn(s_enc, e4m3_value(sf)), FLT_MAX);
         const int64_t gr = r0 / 16 + tr, gc = c0 / 16 + tc;
         if (gr < St && gc < S) {
           if (scales) scales[gr * S + gc] = (uint8_t)sf;

@@ -297,7 +297,9 @@ float orc_amax(const float* x, int64_t n) {
 /* 6 * 448 = 2688: s_enc = RN(2688 / A) (largest finite float if that       */
 /* overflows), s_dec = RN(A / 2688); A = 0 gives s_enc = s_dec = 1.         */
 /* Block: t = RN(RN(b * s_enc) / 6), sf = E4M3(t), inv = RN(s_enc / sf)     */
-/* (0 when sf = 0), element v = RN(x * inv) rounded to E2M1.                */
+/* (0 when sf = 0; the largest finite float if it overflows, which only a   */
+/* block whose max is below ~1.8e-38 can cause), element v = RN(x * inv)    */
+/* rounded to E2M1.                                                         */
 /* ------------------------------------------------------------------------ */
 void orc_nvfp4_global_scales(float A, float* s_enc, float* s_dec) {
   if (A == 0.0f) { *s_enc = 1.0f; *s_dec = 1.0f; return; }
@@ -333,6 +335,7 @@ static void nvfp4_rows_worker(void* p, int64_t r0, int64_t r1) {
       uint8_t sf = orc_e4m3_rne_sat(t);
       float sfv = (float)orc_e4m3_value(sf);
       float inv = (sf == 0) ? 0.0f : q->s_enc / sfv;
+      if (isinf(inv)) inv = FLT_MAX;   /* reading: the reciprocal saturates */
       q->scales[r * nb + b] = sf;
       for (int j = 0; j < 16; ++j) {
         int64_t c = b * 16 + j;
@@ -410,6 +413,7 @@ static void nvfp4_2d_worker(void* p, int64_t t0, int64_t t1) {
       uint8_t sf = orc_e4m3_rne_sat(t);
       float sfv = (float)orc_e4m3_value(sf);
       float inv = (sf == 0) ? 0.0f : q->s_enc / sfv;
+      if (isinf(inv)) inv = FLT_MAX;   /* reading: the reciprocal saturates */
       q->scales[i * tc + j] = sf;
       for (int a = 0; a < 16; ++a)
         for (int b = 0; b < 16; ++b) {

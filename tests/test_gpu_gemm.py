@@ -78,7 +78,7 @@ def test_gemm_bf16_output_and_2d_weights(gpu_lib):
     F.fp4_gemm(ta, tb, out32)
     torch.cuda.synchronize()
     assert rel_fro(out32.cpu().numpy(), ref) <= TOL
-    assert np.array_equal(out.cpu(), out32.to(torch.bfloat16).cpu())
+    assert torch.equal(out.cpu(), out32.to(torch.bfloat16).cpu())
 
 
 def test_gemm_leading_dimension(gpu_lib):

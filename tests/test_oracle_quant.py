@@ -268,3 +268,21 @@ def test_gemm_of_quantized_close_to_unquantized():
     ref = X.astype(np.float64) @ W.T.astype(np.float64)
     rel = np.linalg.norm(y - ref) / np.linalg.norm(ref)
     assert 0.02 < rel < 0.2      # FP4 noise level, not a gross mistake
+
+
+def test_nvfp4_reciprocal_saturates_for_subnormal_blocks():
+    """reading: when s_enc / sf overflows (only a block whose max is below
+    ~1.8e-38 can cause it) the reciprocal is the largest finite float, so a
+    zero stays a zero and nothing becomes NaN or saturates spuriously."""
+    rng = np.random.default_rng(21)
+    x = (rng.standard_normal((4, 64)) * 1e-39).astype(np.float32)
+    x[0, :8] = 0.0
+    x[1, :4] = -0.0
+    q = O.nvfp4_quantize_1d(x)
+    codes = _codes(q["codes"])
+    assert (codes[0, :8] == 0).all() and (codes[1, :4] == 8).all()
+    s_enc, _ = O.nvfp4_global_scales(q["amax"])
+    assert s_enc == np.float32(3.4028235e38)          # 2688 / amax overflowed
+    v = _e2m1(codes)
+    assert np.isfinite(v).all() and (np.abs(v) <= 6).all()
+    assert (np.sign(v[v != 0]) == np.sign(x[v != 0])).all()
