@@ -47,8 +47,9 @@ inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
 fp4_status check_qtensor(const fp4_qtensor* q, int64_t rows, int64_t cols, int32_t fmt,
                          int32_t block) {
-  if (q->codes == nullptr) return FP4_ERR_NULL;
-  if (q->scales == nullptr && q->scales_mma == nullptr) return FP4_ERR_NULL;
+  const bool empty = rows == 0 || cols == 0;   // nothing to encode: buffers may be NULL
+  if (q->codes == nullptr && !empty) return FP4_ERR_NULL;
+  if (q->scales == nullptr && q->scales_mma == nullptr && !empty) return FP4_ERR_NULL;
   if (q->s_dec == nullptr) return FP4_ERR_NULL;
   if (fmt == FP4_NVFP4 && q->amax == nullptr) return FP4_ERR_NULL;
   if (q->rows != rows || q->cols != cols) return FP4_ERR_SHAPE;

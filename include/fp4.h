@@ -83,7 +83,7 @@ enum { FQT_RHT_FPROP = 1, FQT_RHT_DGRAD = 2, FQT_RHT_WGRAD = 4 };
 /* ---------------------------------------------------------------------- */
 /* A quantized operand (all buffers caller-allocated device memory).       */
 /*                                                                         */
-/* codes      [rows, cols/2] bytes.                                        */
+/* codes      [rows, cols/2] bytes (may be NULL for an empty operand).     */
 /* scales     logical block scales, may be NULL:                           */
 /*              NVFP4 1-D: [rows, cols/16] E4M3; NVFP4 2-D: [rows/16,      */
 /*              cols/16] E4M3 (one per 16x16 tile); MXFP4: [rows, cols/32]  */
