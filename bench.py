@@ -56,7 +56,7 @@ def peaks():
 # clocks sampling (nvidia-smi during the timed region)
 # ---------------------------------------------------------------------------
 class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
 
@@ -85,19 +85,25 @@ class ClockSampler:
                 out, _ = self.proc.communicate()
             self.lines = [l for l in out.splitlines() if l.strip()]
 
-    def summary(self):
+    def summary(self, t_start=None, t_end=None):
+        """Median SM clock and active throttle reasons of the samples taken
+        between the wall-clock times t_start and t_end (all if not given)."""
+        import datetime
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for l in getattr(self, "lines", []):
             parts = [p.strip() for p in l.split(",")]
-            if len(parts) < 6:
+            if len(parts) < 7:
                 continue
             try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                if t_start is not None and not (t_start <= ts <= t_end):
+                    continue
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
             except ValueError:
                 continue
-            for n, v in zip(names, parts[2:6]):
+            for n, v in zip(names, parts[3:7]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
         if not sm:
@@ -281,11 +287,13 @@ def run_ours(args, rank, world, device):
     evs = [[(mk(), mk()) for _ in calls] for _ in range(args.steps)]
     launches0 = F.kernel_launches()
     t0, t1 = mk(), mk()
+    wall0 = time.time()
     t0.record()
     for i in range(args.steps):
         step(calls, evs[i])
     t1.record()
     torch.cuda.synchronize()
+    wall1 = time.time()
     clk.__exit__(None, None, None)
     launches = F.kernel_launches() - launches0
     if world > 1:
@@ -350,7 +358,7 @@ def run_ours(args, rank, world, device):
                       "bytes_per_elem": Q_BYTES_PER_ELEM, "launches": q_n,
                       "share_of_step": round(q_ms / (ms_max * args.steps), 3)},
         "gpu_launches": launches,
-        "clocks": clk.summary(),
+        "clocks": clk.summary(wall0, wall1),
     }
     if e2e is not None:
         out["e2e"] = e2e
