@@ -33,7 +33,7 @@ STATUS = {0: "FP4_OK", 1: "FP4_ERR_NULL", 2: "FP4_ERR_SHAPE", 3: "FP4_ERR_ALIGN"
 EXPORTS = ("fp4_qtensor_sizes", "fp4_qparams_default", "fp4_workspace_bytes", "fp4_quantize",
            "fp4_gemm", "fqt_linear_cfg_default", "fqt_linear_fwd", "fqt_linear_bwd",
            "fp4_read_device_status", "fp4_clear_device_status", "fp4_status_str",
-           "fp4_abi_version", "fp4_kernel_launches")
+           "fp4_abi_version", "fp4_kernel_launches", "fp4_gemm_noalloc")
 
 
 class Fp4Error(RuntimeError):
@@ -109,6 +109,9 @@ def load() -> C.CDLL:
     L.fp4_abi_version.argtypes = []
     L.fp4_kernel_launches.restype = C.c_uint64
     L.fp4_kernel_launches.argtypes = []
+    L.fp4_gemm_noalloc.restype = i32
+    L.fp4_gemm_noalloc.argtypes = [C.POINTER(QTensorC), C.POINTER(QTensorC), C.c_float, vp, i64,
+                                   i32, vp, vp]
     _lib = L
     return L
 
@@ -229,6 +232,18 @@ def fp4_gemm(a: QTensor, b: QTensor, out: torch.Tensor, alpha: float = 1.0,
     code = load().fp4_gemm(C.byref(a.c), C.byref(b.c), float(alpha), _ptr(out), out.stride(0), od,
                            _ptr(c_amax), ws.ptr, ws.nbytes, _stream(stream))
     _check(code, "fp4_gemm")
+
+
+def fp4_gemm_noalloc(a: QTensor, b: QTensor, out: torch.Tensor, alpha: float = 1.0,
+                     c_amax: torch.Tensor | None = None, stream=None):
+    """fp4_gemm without a workspace: for callers that cannot allocate device
+    memory.  Its scratch is a small array held by the library on each device;
+    calls that overlap on the GPU share it and race."""
+    assert out.dtype in (torch.bfloat16, torch.float32) and out.is_cuda and out.stride(1) == 1
+    od = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
+    code = load().fp4_gemm_noalloc(C.byref(a.c), C.byref(b.c), float(alpha), _ptr(out),
+                                   out.stride(0), od, _ptr(c_amax), _stream(stream))
+    _check(code, "fp4_gemm_noalloc")
 
 
 def linear_cfg(fmt: int = NVFP4, **overrides) -> LinearCfgC:

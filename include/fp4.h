@@ -220,6 +220,32 @@ fp4_status fqt_linear_bwd(const fqt_linear_cfg* cfg, int64_t M, int64_t N, int64
                           const void* dy, fqt_saved* saved, void* dx, float* dw,
                           void* ws, size_t ws_bytes, void* stream);
 
+/* fp4_gemm for callers that cannot allocate device memory (no counterpart
+ * in the paper; an addition of this library).
+ *
+ * fp4_gemm needs a caller-allocated workspace, which the GEMM uses as scratch
+ * for its device status block.  Callers that cannot call cudaMalloc -- code
+ * running while a framework's pool or arena owns all device memory, plugins
+ * in host processes that forbid device allocation, paths that must not risk
+ * the synchronisation cudaMalloc can cause -- use this entry point instead.
+ * Its scratch is a static device array inside the library of
+ * FP4_NOALLOC_SCRATCH_BYTES bytes per device, held by every GPU that loads
+ * the library until the process exits.  Same arguments and results as
+ * fp4_gemm, without `ws`; inputs and outputs are still caller-provided.
+ *   - Problems whose workspace need (fp4_workspace_bytes(M, N, K)) exceeds
+ *     FP4_NOALLOC_SCRATCH_BYTES are rejected with FP4_ERR_WORKSPACE.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before any
+ *     stream capture.
+ *   - Every call shares the one array: each call clears its status block on
+ *     `stream` first, and calls that overlap on the GPU (other streams, other
+ *     threads) race on it.  Device conditions of a call are not reported
+ *     through this entry point; callers that need them use fp4_gemm. */
+#define FP4_NOALLOC_SCRATCH_BYTES 4096
+fp4_status fp4_gemm_noalloc(const fp4_qtensor* a, const fp4_qtensor* b, float alpha, void* c,
+                            int64_t ldc, int32_t out_dtype, float* c_amax, void* stream);
+
 /* Synchronise `stream`, then return the device status word of `ws`
  * (FP4_OK when no device condition was recorded). */
 fp4_status fp4_read_device_status(const void* ws, void* stream);
