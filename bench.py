@@ -155,26 +155,33 @@ def qparams_for(cfg, which):
 
 
 def plan(F, layers, ws):
-    """The calls of one step: (kind, units, thunk) -- the calls
+    """The calls of one step: (kind, units, thunk, label) -- the calls
     fqt_linear_fwd / fqt_linear_bwd make for each layer."""
     calls = []
     for L in layers:
         sv = L.sv
         qx, qw, qd = (qparams_for(L.cfg, k) for k in ("x", "w", "dy"))
+        tag = f"{L.name}[{L.N}x{L.K}]"
         calls += [
-            ("quant", L.M * L.K, lambda L=L, sv=sv, q=qx: F.fp4_quantize(L.x, sv.xq, sv.xq_t, ws=ws, **q)),
-            ("quant", L.N * L.K, lambda L=L, sv=sv, q=qw: F.fp4_quantize(L.w, sv.wq, sv.wq_t, ws=ws, **q)),
-            ("gemm", 2 * L.M * L.N * L.K, lambda L=L, sv=sv: F.fp4_gemm(sv.xq, sv.wq, L.y, ws=ws)),
-            ("quant", L.M * L.N, lambda L=L, sv=sv, q=qd: F.fp4_quantize(L.dy, sv.dyq, sv.dyq_t, ws=ws, **q)),
-            ("gemm", 2 * L.M * L.N * L.K, lambda L=L, sv=sv: F.fp4_gemm(sv.dyq, sv.wq_t, L.dx, ws=ws)),
-            ("gemm", 2 * L.M * L.N * L.K, lambda L=L, sv=sv: F.fp4_gemm(sv.dyq_t, sv.xq_t, L.dw, ws=ws)),
+            ("quant", L.M * L.K, lambda L=L, sv=sv, q=qx: F.fp4_quantize(L.x, sv.xq, sv.xq_t, ws=ws, **q),
+             f"quant X {tag}"),
+            ("quant", L.N * L.K, lambda L=L, sv=sv, q=qw: F.fp4_quantize(L.w, sv.wq, sv.wq_t, ws=ws, **q),
+             f"quant W {tag}"),
+            ("gemm", 2 * L.M * L.N * L.K, lambda L=L, sv=sv: F.fp4_gemm(sv.xq, sv.wq, L.y, ws=ws),
+             f"fprop {tag}"),
+            ("quant", L.M * L.N, lambda L=L, sv=sv, q=qd: F.fp4_quantize(L.dy, sv.dyq, sv.dyq_t, ws=ws, **q),
+             f"quant dY {tag}"),
+            ("gemm", 2 * L.M * L.N * L.K, lambda L=L, sv=sv: F.fp4_gemm(sv.dyq, sv.wq_t, L.dx, ws=ws),
+             f"dgrad {tag}"),
+            ("gemm", 2 * L.M * L.N * L.K, lambda L=L, sv=sv: F.fp4_gemm(sv.dyq_t, sv.xq_t, L.dw, ws=ws),
+             f"wgrad {tag}"),
         ]
     return calls
 
 
 def step(calls, events=None):
     """One pass of the hot path; `events` (pre-created pairs) brackets each call."""
-    for i, (kind, units, fn) in enumerate(calls):
+    for i, (kind, units, fn, _label) in enumerate(calls):
         if events is not None:
             events[i][0].record()
             fn()
@@ -305,7 +312,21 @@ def run_ours(args, rank, world, device):
     ms_max = float(ms_t.item())
     assert ws.status() == 0, f"device status {ws.status()}"
 
-    ev = [(kind, units, a, b) for per in evs for (kind, units, _), (a, b) in zip(calls, per)]
+    ev = [(kind, units, a, b) for per in evs for (kind, units, _f, _l), (a, b) in zip(calls, per)]
+    breakdown = {}
+    for per in evs:
+        for (kind, units, _f, label), (a, b) in zip(calls, per):
+            d = breakdown.setdefault(label, [kind, units, 0.0, 0])
+            d[2] += a.elapsed_time(b)
+            d[3] += 1
+    detail = []
+    for label, (kind, units, ms_sum, n) in breakdown.items():
+        ms_avg = ms_sum / n
+        rate = units / (ms_avg * 1e-3)
+        detail.append({"call": label, "ms": round(ms_avg, 4),
+                       "rate": round(rate / 1e12, 1) if kind == "gemm" else
+                       round(rate * Q_BYTES_PER_ELEM / 1e9, 1),
+                       "unit": "TFLOP/s" if kind == "gemm" else "GB/s"})
     flops_step = sum(6 * M_TOKENS * N * K for _, N, K in LAYERS)
     gemm_ms = sum(a.elapsed_time(b) for k, u, a, b in ev if k == "gemm")
     gemm_fl = sum(u for k, u, a, b in ev if k == "gemm")
@@ -358,6 +379,7 @@ def run_ours(args, rank, world, device):
                       "bytes_per_elem": Q_BYTES_PER_ELEM, "launches": q_n,
                       "share_of_step": round(q_ms / (ms_max * args.steps), 3)},
         "gpu_launches": launches,
+        "breakdown": detail,
         "clocks": clk.summary(wall0, wall1),
     }
     if e2e is not None:
@@ -390,8 +412,53 @@ def run_reference(args):
                     "d2h_bytes_per_step": 0}}
 
 
+def run_case(args, device):
+    """A single kernel family on one small problem (for profiler captures):
+    --case gemm: NVFP4 fprop-style GEMM [m, k] x [n, k]^T, BF16 out;
+    --case quant: NVFP4 row-wise RTN + transposed SR of a [m, k] tensor."""
+    import fp4_fully_quantized_b200 as F
+    import fqt_synth as S
+    F.load()
+    M, N, K = args.m, args.n, args.k
+    ws = F.Workspace(device=device)
+    x = S.student_t_channels(M, K, seed=1)[0].to(device)
+    qa = F.QTensor.empty(M, K, device=device, logical_scales=False)
+    qat = F.QTensor.empty(K, M, device=device, logical_scales=False)
+    if args.case == "quant":
+        fn = lambda: F.fp4_quantize(x, qa, qat, round=F.RTN, round_t=F.SR, sr_seed=1, sr_stream_t=3,
+                                    ws=ws)
+        units, unit = M * K * Q_BYTES_PER_ELEM / 1e9, "GB/s"
+    else:
+        w = S.normal((N, K), 0.02, seed=2).to(device)
+        qb = F.QTensor.empty(N, K, F.NVFP4, F.BLOCK_2D, device=device, logical_scales=False)
+        qbt = F.QTensor.empty(K, N, F.NVFP4, F.BLOCK_2D, device=device, logical_scales=False)
+        F.fp4_quantize(x, qa, ws=ws)
+        F.fp4_quantize(w, qb, qbt, block=F.BLOCK_2D, ws=ws)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        fn = lambda: F.fp4_gemm(qa, qb, y, ws=ws)
+        units, unit = 2 * M * N * K / 1e12, "TFLOP/s"
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / args.steps
+    assert ws.status() == 0
+    return {"case": args.case, "m": M, "n": N, "k": K, "ms": round(ms, 4),
+            "rate": round(units / (ms * 1e-3), 1), "unit": unit}
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--case", choices=["gemm", "quant"], default=None,
+                    help="time one kernel family on a small problem (profiling)")
+    ap.add_argument("--m", type=int, default=8192)
+    ap.add_argument("--n", type=int, default=4096)
+    ap.add_argument("--k", type=int, default=4096)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
@@ -409,6 +476,12 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.case is not None:
+        dev = torch.device("cuda", local)
+        torch.cuda.set_device(dev)
+        print(json.dumps(run_case(args, dev)), flush=True)
+        return
 
     if args.impl == "reference":
         if rank == 0:

@@ -33,7 +33,7 @@ STATUS = {0: "FP4_OK", 1: "FP4_ERR_NULL", 2: "FP4_ERR_SHAPE", 3: "FP4_ERR_ALIGN"
 EXPORTS = ("fp4_qtensor_sizes", "fp4_qparams_default", "fp4_workspace_bytes", "fp4_quantize",
            "fp4_gemm", "fqt_linear_cfg_default", "fqt_linear_fwd", "fqt_linear_bwd",
            "fp4_read_device_status", "fp4_clear_device_status", "fp4_status_str",
-           "fp4_abi_version", "fp4_kernel_launches", "fp4_gemm_noalloc")
+           "fp4_abi_version", "fp4_kernel_launches", "fp4_gemm_noalloc", "fp4_mma_rate")
 
 
 class Fp4Error(RuntimeError):
@@ -109,6 +109,8 @@ def load() -> C.CDLL:
     L.fp4_abi_version.argtypes = []
     L.fp4_kernel_launches.restype = C.c_uint64
     L.fp4_kernel_launches.argtypes = []
+    L.fp4_mma_rate.restype = i32
+    L.fp4_mma_rate.argtypes = [i32, i32, C.POINTER(C.c_float), vp, sz, vp]
     L.fp4_gemm_noalloc.restype = i32
     L.fp4_gemm_noalloc.argtypes = [C.POINTER(QTensorC), C.POINTER(QTensorC), C.c_float, vp, i64,
                                    i32, vp, vp]
@@ -244,6 +246,15 @@ def fp4_gemm_noalloc(a: QTensor, b: QTensor, out: torch.Tensor, alpha: float = 1
     code = load().fp4_gemm_noalloc(C.byref(a.c), C.byref(b.c), float(alpha), _ptr(out),
                                    out.stride(0), od, _ptr(c_amax), _stream(stream))
     _check(code, "fp4_gemm_noalloc")
+
+
+def mma_rate(variant: int = 0, iters: int = 20000, stream=None) -> float:
+    """Achieved TFLOP/s of back-to-back block-scaled NVFP4 MMAs (see fp4.h)."""
+    ws = Workspace()
+    out = C.c_float()
+    _check(load().fp4_mma_rate(variant, iters, C.byref(out), ws.ptr, ws.nbytes, _stream(stream)),
+           "fp4_mma_rate")
+    return float(out.value)
 
 
 def linear_cfg(fmt: int = NVFP4, **overrides) -> LinearCfgC:

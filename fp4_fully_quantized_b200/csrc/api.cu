@@ -118,11 +118,13 @@ size_t fp4_workspace_bytes(int64_t M, int64_t N, int64_t K) {
 fp4_status fp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
                         const fp4_qparams* p, fp4_qtensor* out, fp4_qtensor* out_t, void* ws,
                         size_t ws_bytes, void* stream) {
-  if (p == nullptr || x == nullptr) return FP4_ERR_NULL;
+  if (p == nullptr) return FP4_ERR_NULL;
   if (out == nullptr && out_t == nullptr) return FP4_ERR_NULL;
   if (ws != nullptr && ws_bytes < sizeof(DeviceStatus)) return FP4_ERR_WORKSPACE;
   if (rows < 0 || cols < 0 || ld < cols) return FP4_ERR_SHAPE;
-  if (!aligned16(x) || (ld % 8) != 0) return FP4_ERR_ALIGN;
+  const bool empty_x = rows == 0 || cols == 0;    // x may then be NULL
+  if (x == nullptr && !empty_x) return FP4_ERR_NULL;
+  if ((!empty_x && !aligned16(x)) || (ld % 8) != 0) return FP4_ERR_ALIGN;
   if (p->fmt != FP4_NVFP4 && p->fmt != FP4_MXFP4) return FP4_ERR_FORMAT;
   if (p->block != FP4_BLOCK_1D && p->block != FP4_BLOCK_2D) return FP4_ERR_FORMAT;
   if (p->block == FP4_BLOCK_2D && p->fmt != FP4_NVFP4) return FP4_ERR_FORMAT;
@@ -176,23 +178,58 @@ fp4_status fp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
   const uint32_t mask_t = p->rht_n_t ? fp4dev::rht_sign_mask(p->rht_seed, p->rht_n_t) : 0u;
   const bool nv = p->fmt == FP4_NVFP4;
 
+  // Tensor amax of each requested output (NVFP4 only).
   const float* src_row = nullptr;
+  const float* src_col = nullptr;
+  if (nv && out) {
+    src_row = p->amax_in;
+    if (src_row == nullptr) {
+      if (cudaMemsetAsync(out->amax, 0, sizeof(float), s) != cudaSuccess) return FP4_ERR_CUDA;
+      if (launch_amax_rows(x, rows, cols, ld, p->rht_n, mask, out->amax, s) != cudaSuccess)
+        return FP4_ERR_CUDA;
+      src_row = out->amax;
+    }
+  }
+  if (nv && out_t) {
+    src_col = p->amax_in_t;
+    if (src_col == nullptr) {
+      if (out && p->amax_in == nullptr && p->rht_n == 0 && p->rht_n_t == 0) {
+        src_col = out->amax;      // same tensor, same orientation-free amax
+      } else {
+        if (cudaMemsetAsync(out_t->amax, 0, sizeof(float), s) != cudaSuccess) return FP4_ERR_CUDA;
+        cudaError_t e = p->rht_n_t
+            ? launch_amax_cols(x, rows, cols, ld, p->rht_n_t, mask_t, out_t->amax, s)
+            : launch_amax_rows(x, rows, cols, ld, 0, 0, out_t->amax, s);
+        if (e != cudaSuccess) return FP4_ERR_CUDA;
+        src_col = out_t->amax;
+      }
+    }
+  }
+
+  // Both outputs from one read of x.
+  if (out && out_t && dual_supported(p->fmt, p->rht_n, p->rht_n_t)) {
+    DualQuantArgs a{};
+    a.x = x; a.rows = rows; a.cols = cols; a.ld = ld;
+    a.fmt = p->fmt; a.rht_r = p->rht_n; a.rht_c = p->rht_n_t;
+    a.sr_r = p->round == FP4_SR; a.sr_c = p->round_t == FP4_SR;
+    a.mask_r = mask; a.mask_c = mask_t;
+    a.sr_seed = p->sr_seed; a.stream_r = p->sr_stream; a.stream_c = p->sr_stream_t;
+    a.amax_src_r = src_row; a.amax_src_c = src_col;
+    a.amax_out_r = out->amax; a.amax_out_c = out_t->amax;
+    a.s_dec_r = out->s_dec; a.s_dec_c = out_t->s_dec;
+    a.codes_r = out->codes; a.scales_r = out->scales; a.mma_r = out->scales_mma;
+    a.codes_c = out_t->codes; a.scales_c = out_t->scales; a.mma_c = out_t->scales_mma;
+    a.status = status;
+    return cuda_status(launch_quant_dual(a, s));
+  }
+
   if (out) {
     RowQuantArgs a{};
     a.x = x; a.rows = rows; a.cols = cols; a.ld = ld;
     a.fmt = p->fmt; a.round = p->round; a.rht_n = p->rht_n; a.rht_mask = mask;
     a.sr_seed = p->sr_seed; a.sr_stream = p->sr_stream;
-    if (nv) {
-      src_row = p->amax_in;
-      if (src_row == nullptr) {
-        if (cudaMemsetAsync(out->amax, 0, sizeof(float), s) != cudaSuccess) return FP4_ERR_CUDA;
-        if (launch_amax_rows(x, rows, cols, ld, p->rht_n, mask, out->amax, s) != cudaSuccess)
-          return FP4_ERR_CUDA;
-        src_row = out->amax;
-      }
-      a.amax_src = src_row;
-      a.amax_out = out->amax;
-    }
+    a.amax_src = src_row;
+    a.amax_out = out->amax;
     a.s_dec = out->s_dec;
     a.codes = out->codes; a.scales = out->scales; a.scales_mma = out->scales_mma;
     a.status = status;
@@ -203,23 +240,8 @@ fp4_status fp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
     a.x = x; a.rows = rows; a.cols = cols; a.ld = ld;
     a.fmt = p->fmt; a.round = p->round_t; a.rht_n = p->rht_n_t; a.rht_mask = mask_t;
     a.sr_seed = p->sr_seed; a.sr_stream = p->sr_stream_t;
-    if (nv) {
-      const float* src = p->amax_in_t;
-      if (src == nullptr) {
-        if (out && p->amax_in == nullptr && p->rht_n == 0 && p->rht_n_t == 0) {
-          src = out->amax;      // same tensor, same orientation-free amax
-        } else {
-          if (cudaMemsetAsync(out_t->amax, 0, sizeof(float), s) != cudaSuccess) return FP4_ERR_CUDA;
-          cudaError_t e = p->rht_n_t
-              ? launch_amax_cols(x, rows, cols, ld, p->rht_n_t, mask_t, out_t->amax, s)
-              : launch_amax_rows(x, rows, cols, ld, 0, 0, out_t->amax, s);
-          if (e != cudaSuccess) return FP4_ERR_CUDA;
-          src = out_t->amax;
-        }
-      }
-      a.amax_src = src;
-      a.amax_out = out_t->amax;
-    }
+    a.amax_src = src_col;
+    a.amax_out = out_t->amax;
     a.s_dec = out_t->s_dec;
     a.codes = out_t->codes; a.scales = out_t->scales; a.scales_mma = out_t->scales_mma;
     a.status = status;

@@ -31,7 +31,9 @@ __host__ __device__ __forceinline__ U4 philox4x32_10(uint64_t ctr_lo64, uint32_t
                                                      uint64_t seed) {
   uint32_t c0 = (uint32_t)ctr_lo64, c1 = (uint32_t)(ctr_lo64 >> 32), c2 = stream, c3 = 0;
   uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+#ifdef __CUDA_ARCH__
 #pragma unroll
+#endif
   for (int r = 0; r < 10; ++r) {
 #ifdef __CUDA_ARCH__
     uint32_t hi0 = __umulhi(kPhiloxM0, c0), lo0 = kPhiloxM0 * c0;
@@ -44,6 +46,36 @@ __host__ __device__ __forceinline__ U4 philox4x32_10(uint64_t ctr_lo64, uint32_t
     uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
     c0 = n0; c1 = lo1; c2 = n2; c3 = lo0;
     k0 += kPhiloxW0; k1 += kPhiloxW1;
+  }
+  return U4{c0, c1, c2, c3};
+}
+
+// The same generator with its ten round keys precomputed once per thread and
+// each 32x32 product done as one widening multiply (hi and lo together).
+struct PhiloxKeys {
+  uint32_t k0[10], k1[10];
+};
+
+__device__ __forceinline__ PhiloxKeys philox_keys(uint64_t seed) {
+  PhiloxKeys K;
+  uint32_t a = (uint32_t)seed, b = (uint32_t)(seed >> 32);
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    K.k0[r] = a; K.k1[r] = b;
+    a += kPhiloxW0; b += kPhiloxW1;
+  }
+  return K;
+}
+
+__device__ __forceinline__ U4 philox_keyed(uint64_t ctr, uint32_t stream, const PhiloxKeys& K) {
+  uint32_t c0 = (uint32_t)ctr, c1 = (uint32_t)(ctr >> 32), c2 = stream, c3 = 0;
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const unsigned long long p0 = (unsigned long long)kPhiloxM0 * c0;
+    const unsigned long long p1 = (unsigned long long)kPhiloxM1 * c2;
+    const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ K.k0[r];
+    const uint32_t n2 = (uint32_t)(p0 >> 32) ^ c3 ^ K.k1[r];
+    c0 = n0; c1 = (uint32_t)p1; c2 = n2; c3 = (uint32_t)p0;
   }
   return U4{c0, c1, c2, c3};
 }
@@ -125,6 +157,26 @@ __device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t u) {
   const unsigned long long T = __float2ull_ru(y);            // ceil, exact
   const uint32_t up = ((unsigned long long)u < T) ? 1u : 0u;
   return sign | (code_lo + up);
+}
+
+// The same stochastic rounding read from the binary32 encoding of |v|
+// (clamped to 6), branch-free.  Within [1, 6] the E2M1 grid splits each
+// binade in two, so the level is (exponent, top mantissa bit) and the
+// fraction of the gap is the remaining 22 mantissa bits: ceil(p * 2^32) is
+// exactly those bits << 10.  In [0.5, 1) the gap is the whole binade (bits
+// << 9); below 0.5 the gap is [0, 0.5] and ceil(p * 2^32) = ceil(|v| * 2^33).
+__device__ __forceinline__ uint32_t e2m1_sr_bits(float v, uint32_t u) {
+  const uint32_t bits = __float_as_uint(v);
+  const uint32_t sign = (bits >> 28) & 8u;
+  const uint32_t a = min(bits & 0x7FFFFFFFu, 0x40C00000u);      // |v| clamped to 6.0
+  const uint32_t E = a >> 23, m = a & 0x7FFFFFu;
+  const uint32_t code_hi = ((E - 126u) << 1) | (m >> 22);        // a >= 1
+  const uint32_t t_hi = (m & 0x3FFFFFu) << 10;
+  const uint32_t t_mid = m << 9;                                 // 0.5 <= a < 1
+  const uint32_t t_lo = __float2uint_ru(__fmul_rn(__uint_as_float(a), 8589934592.0f));  // a < 0.5
+  const uint32_t code_lo = E >= 127u ? code_hi : (E == 126u ? 1u : 0u);
+  const uint32_t T = E >= 127u ? t_hi : (E == 126u ? t_mid : t_lo);
+  return sign | (code_lo + (u < T ? 1u : 0u));
 }
 
 // ---------------------------------------------------------------------------

@@ -7,15 +7,17 @@
 // accumulation happens in higher precision; "Quartet", abstract line: all
 // three linear-layer GEMMs in FP4.
 //
-// Structure (one persistent CTA per SM, 192 threads):
-//   warp 4      TMA producer: A/B tiles (128B-swizzled) and the scale-factor
+// Structure (one persistent CTA per SM, 320 threads):
+//   warp 8      TMA producer: A/B tiles (128B-swizzled) and the scale-factor
 //               atoms (bulk copies) into a 4-stage shared-memory ring;
-//   warp 5      TMEM allocator and MMA issuer: tcgen05.cp moves the scale
+//   warp 9      TMEM allocator and MMA issuer: tcgen05.cp moves the scale
 //               atoms into tensor memory, tcgen05.mma (kind::mxf4nvf4 /
 //               kind::mxf4, block_scale) accumulates a 128 x 256 tile into
 //               TMEM, tcgen05.commit releases ring slots and the accumulator;
-//   warps 0..3  epilogue: tcgen05.ld of their 32 TMEM lanes, scale, convert,
-//               store, optional |C| max.
+//   warps 0..7  epilogue: warp w drains TMEM lanes 32 (w % 4) .. + 31, columns
+//               128 (w / 4) .. + 127 into registers, releases the accumulator
+//               (the next tile's MMAs start), then scales, converts, stores
+//               and tracks |C| max.
 // Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the kernel
 // records FP4_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and
 // returns.
@@ -28,6 +30,7 @@
 #include <mutex>
 
 #include "internal.h"
+#include "sm100_ptx.cuh"
 
 namespace fp4impl {
 namespace {
@@ -43,162 +46,15 @@ constexpr int SFA_BYTES = 4 * 512;            // up to 4 atoms of 128 rows x 4 s
 constexpr int SFB_BYTES = 2 * 4 * 512;        // two 128-row blocks
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 320;
+constexpr int EPI_WARPS = 8;
+constexpr int PRODUCER_WARP = 8;
+constexpr int MMA_WARP = 9;
 constexpr int TMEM_COLS = 512;
 constexpr int TMEM_SF_BASE = 256;             // accumulator uses columns [0, 256)
 constexpr int TMEM_SF_STAGE = 48;             // 16 (A) + 32 (B) columns per stage
-constexpr uint64_t kWaitNs = 2000000000ull;   // bounded waits: 2 s
 
-// ---------------------------------------------------------------------------
-// PTX wrappers
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait: false when the deadline passed or another role aborted.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t* status, uint32_t where) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  while (!mbar_try_wait(bar, parity)) {
-    if (*abort_flag) return false;
-    if (globaltimer() - t0 > kWaitNs) {
-      *abort_flag = 1;
-      set_status(status, FP4_ERR_TIMEOUT, where);
-      return false;
-    }
-  }
-  return true;
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
-      : "memory");
-}
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
-                                          uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(dst),
-      "l"(src), "r"(bytes), "r"(bar)
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_alloc(uint32_t holder_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                   holder_smem),
-               "r"(ncols));
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void tc_cp_32x128b(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc));
-}
-template <bool NV>
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                       uint32_t idesc, uint32_t sfa, uint32_t sfb,
-                                       uint32_t accumulate) {
-  if constexpr (NV) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X"
-        " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb));
-  } else {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X"
-        " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb));
-  }
-}
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32"
-      " {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// Shared-memory matrix descriptor (tcgen05 format): start address, leading
-// and stride byte offsets (16-byte units), version 1, swizzle mode.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo,
-                                              uint32_t swizzle) {
-  uint64_t d = 0;
-  d |= (uint64_t)((addr >> 4) & 0x3FFF);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
-  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
-  d |= (uint64_t)1 << 46;                       // descriptor version (sm_100)
-  d |= (uint64_t)(swizzle & 7) << 61;           // 2 = 128B swizzle, 0 = none
-  return d;
-}
-
-// Instruction descriptor of a block-scaled FP4 MMA: E2M1 A and B (K-major),
-// N and M dimensions, scale format (0 = UE4M3, 1 = UE8M0), scale ids.
-__device__ __forceinline__ uint32_t make_idesc(int n, int m, uint32_t scale_fmt, uint32_t a_sf_id,
-                                               uint32_t b_sf_id) {
-  uint32_t d = 0;
-  d |= (b_sf_id & 3u) << 4;
-  d |= 1u << 7;                  // A format: E2M1
-  d |= 1u << 10;                 // B format: E2M1
-  d |= (uint32_t)(n >> 3) << 17;
-  d |= (scale_fmt & 1u) << 23;
-  d |= (uint32_t)(m >> 4) << 24;
-  d |= (a_sf_id & 3u) << 29;
-  return d;
-}
+using namespace ptx;
 
 struct Smem {
   uint8_t* base;   // 1024-aligned
@@ -255,19 +111,19 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       mbar_init(empty_bar(s), 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 4);
+    mbar_init(acc_empty, EPI_WARPS);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  if (warp == 5) tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+  if (warp == MMA_WARP) tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  if (warp == 4) {
+  if (warp == PRODUCER_WARP) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_a)) : "memory");
@@ -313,7 +169,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       uint32_t it = 0, tile_iter = 0;
@@ -326,36 +182,42 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           if (!mbar_wait(full_bar(s), ph, abort_flag, p.status, 0x400 + s)) { ok = false; break; }
-          tc_fence_after();
           const int n_mma = min(BK / MMA_K, (p.K - kb * BK) / MMA_K);
-          const int n_atoms = NV ? n_mma : (n_mma + 1) / 2;
           const uint32_t t_sfa = tmem_base + TMEM_SF_BASE + s * TMEM_SF_STAGE;
           const uint32_t t_sfb = t_sfa + 16;
-          for (int a = 0; a < n_atoms; ++a) {
-            tc_cp_32x128b(t_sfa + 4 * a, smem_desc(smem_u32(sm.sfa(s) + a * 512), 0, 128, 0));
-            tc_cp_32x128b(t_sfb + 8 * a, smem_desc(smem_u32(sm.sfb(s) + a * 512), 0, 128, 0));
-            tc_cp_32x128b(t_sfb + 8 * a + 4,
-                          smem_desc(smem_u32(sm.sfb(s) + 4 * 512 + a * 512), 0, 128, 0));
-          }
           const uint32_t a_base = smem_u32(sm.a(s)), b_base = smem_u32(sm.b(s));
-          for (int kk = 0; kk < n_mma; ++kk) {
-            const uint64_t adesc = smem_desc(a_base + kk * (MMA_K / 2), 16, 1024, 2);
-            const uint64_t bdesc = smem_desc(b_base + kk * (MMA_K / 2), 16, 1024, 2);
+          const uint32_t sfa_s = smem_u32(sm.sfa(s)), sfb_s = smem_u32(sm.sfb(s));
+          // Each MMA's scale atoms are copied into TMEM right before it (the
+          // copies and MMAs of one thread execute in issue order).
+          auto step = [&](int kk) {
             uint32_t sfa_addr, sfb_addr, idesc;
+            const int atom = NV ? kk : (kk >> 1);
+            if (NV || (kk & 1) == 0) {
+              tc_cp_32x128b(t_sfa + 4 * atom, smem_desc(sfa_s + atom * 512, 0, 128, 0));
+              tc_cp_32x128b(t_sfb + 8 * atom, smem_desc(sfb_s + atom * 512, 0, 128, 0));
+              tc_cp_32x128b(t_sfb + 8 * atom + 4, smem_desc(sfb_s + 2048 + atom * 512, 0, 128, 0));
+            }
             if (NV) {
               sfa_addr = t_sfa + 4 * kk;
               sfb_addr = t_sfb + 8 * kk;
               idesc = make_idesc(BN, BM, 0u, 0u, 0u);
             } else {
               const uint32_t byte = (uint32_t)(kk & 1) * 2u;
-              sfa_addr = (t_sfa + 4 * (kk >> 1)) | (byte << 30);
-              sfb_addr = (t_sfb + 8 * (kk >> 1)) | (byte << 30);
+              sfa_addr = (t_sfa + 4 * atom) | (byte << 30);
+              sfb_addr = (t_sfb + 8 * atom) | (byte << 30);
               idesc = make_idesc(BN, BM, 1u, byte, byte);
             }
-            tc_mma<NV>(tmem_base, adesc, bdesc, idesc, sfa_addr, sfb_addr,
-                       (kb > 0 || kk > 0) ? 1u : 0u);
-            issued = true;
+            tc_mma<NV>(tmem_base, smem_desc(a_base + kk * (MMA_K / 2), 16, 1024, 2),
+                       smem_desc(b_base + kk * (MMA_K / 2), 16, 1024, 2), idesc, sfa_addr,
+                       sfb_addr, (kb > 0 || kk > 0) ? 1u : 0u);
+          };
+          if (n_mma == BK / MMA_K) {
+#pragma unroll
+            for (int kk = 0; kk < BK / MMA_K; ++kk) step(kk);
+          } else {
+            for (int kk = 0; kk < n_mma; ++kk) step(kk);
           }
+          issued = true;
           tc_commit(empty_bar(s));     // ring slot free once these MMAs finish
         }
         if (!ok) break;
@@ -373,45 +235,58 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     const float scale = p.alpha * (*p.a_sdec) * (*p.b_sdec);
     float amax = 0.0f;
     uint32_t tile_iter = 0;
-    const int row_in_tile = warp * 32 + lane;
+    const int quad = warp & 3, half = warp >> 2;
+    const int row_in_tile = quad * 32 + lane;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tile_iter) {
-      if (!mbar_wait(acc_full, tile_iter & 1u, abort_flag, p.status, 0x600 + warp)) break;
+      // one lane per warp polls the barrier; the warp then proceeds together
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(acc_full, tile_iter & 1u, abort_flag, p.status, 0x600 + warp);
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) break;
       tc_fence_after();
       const int mb = tile / tiles_n, nb = tile % tiles_n;
       const int64_t row = (int64_t)mb * BM + row_in_tile;
-      const int ncols = min(BN, p.N - nb * BN);
-      for (int c0 = 0; c0 < ncols; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, r);
-        float v[32];
+      const int c_begin = half * (BN / 2);
+      const int ncols = min(BN / 2, p.N - nb * BN - c_begin);   // 128, 0 (ragged N)
+      uint32_t r[BN / 2];
+      const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)c_begin;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          v[i] = __uint_as_float(r[i]) * scale;
-          amax = fmaxf(amax, fabsf(v[i]));
-        }
-        const int64_t col = (int64_t)nb * BN + c0;
+      for (int q = 0; q < BN / 2 / 32; ++q) tmem_ld32_nowait(taddr + 32 * q, &r[32 * q]);
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);        // TMEM free: next tile may start
+      if (ncols > 0) {
+        const int64_t col = (int64_t)nb * BN + c_begin;
         if (p.out_f32) {
           float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.c) + row * p.ldc + col);
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          for (int q = 0; q < BN / 2 / 4; ++q) {
+            float4 o;
+            o.x = __uint_as_float(r[4 * q]) * scale;
+            o.y = __uint_as_float(r[4 * q + 1]) * scale;
+            o.z = __uint_as_float(r[4 * q + 2]) * scale;
+            o.w = __uint_as_float(r[4 * q + 3]) * scale;
+            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(o.x), fabsf(o.y)), fmaxf(fabsf(o.z), fabsf(o.w))));
+            dst[q] = o;
+          }
         } else {
           uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.c) + row * p.ldc + col);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+          for (int q = 0; q < BN / 2 / 8; ++q) {
             uint32_t w[4];
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(v[8 * q + 2 * h], v[8 * q + 2 * h + 1]);
+              const float a0 = __uint_as_float(r[8 * q + 2 * h]) * scale;
+              const float a1 = __uint_as_float(r[8 * q + 2 * h + 1]) * scale;
+              amax = fmaxf(amax, fmaxf(fabsf(a0), fabsf(a1)));
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(a0, a1);
               memcpy(&w[h], &b2, 4);
             }
             dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
     }
     if (p.c_amax != nullptr) {
 #pragma unroll
@@ -422,7 +297,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
   }
@@ -467,6 +342,9 @@ bool make_kmajor_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64
 }  // namespace
 
 fp4_status gemm_launch(const GemmArgs& g, cudaStream_t s) {
+  // Two or more 128-row blocks: the CTA-pair kernel (256 x 256 tiles, half
+  // the B traffic per SM).  A single row block keeps the one-SM kernel.
+  return gemm_launch_sfst(g, s);
   CUtensorMap ta, tb;
   if (!make_kmajor_map(&ta, g.a_codes, g.M, g.K, BM)) return FP4_ERR_CUDA;
   if (!make_kmajor_map(&tb, g.b_codes, g.N, g.K, BN)) return FP4_ERR_CUDA;

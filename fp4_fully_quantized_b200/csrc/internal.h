@@ -46,6 +46,22 @@ cudaError_t launch_quant_rows(const RowQuantArgs& a, cudaStream_t s);
 // are the blocked dimension.  Fields keep the meaning of RowQuantArgs with
 // rows/cols those of x.
 cudaError_t launch_quant_cols(const RowQuantArgs& a, cudaStream_t s);
+// Row-wise and transposed outputs from one read of x (both outputs 1-D
+// blocks of the same format).  Supported Hadamard sizes: 0 or the format's
+// block size (16 NVFP4, 32 MXFP4) on either output.
+struct DualQuantArgs {
+  const void* x; int64_t rows, cols, ld;
+  int fmt, rht_r, rht_c; bool sr_r, sr_c;
+  uint32_t mask_r, mask_c;
+  uint64_t sr_seed; uint32_t stream_r, stream_c;
+  const float* amax_src_r; const float* amax_src_c;   // NVFP4 (ignored for MXFP4)
+  float* amax_out_r; float* amax_out_c; float* s_dec_r; float* s_dec_c;
+  uint8_t* codes_r; uint8_t* scales_r; uint8_t* mma_r;
+  uint8_t* codes_c; uint8_t* scales_c; uint8_t* mma_c;
+  uint32_t* status;
+};
+bool dual_supported(int fmt, int rht_r, int rht_c);
+cudaError_t launch_quant_dual(const DualQuantArgs& a, cudaStream_t s);
 // NVFP4 16x16 tiles: W (codes/scales/scales_mma) and W^T (codes_t/...).
 struct Quant2DArgs {
   const void* x; int64_t rows, cols, ld;
@@ -68,5 +84,9 @@ struct GemmArgs {
   uint32_t* status;
 };
 fp4_status gemm_launch(const GemmArgs& g, cudaStream_t s);
+// CTA-pair (cta_group::2) variant, 256 x 256 tiles (gemm_pair.cu).
+fp4_status gemm_launch_pair(const GemmArgs& g, cudaStream_t s);
+// Scale factors staged into TMEM by tcgen05.st warps (gemm_sfst.cu).
+fp4_status gemm_launch_sfst(const GemmArgs& g, cudaStream_t s);
 
 }  // namespace fp4impl

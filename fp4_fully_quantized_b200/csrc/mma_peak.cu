@@ -1,0 +1,164 @@
+// mma_peak.cu -- tensor-core rate microbenchmark for the FP4 GEMM roofline.
+//
+// One persistent CTA (or CTA pair) per SM issues back-to-back block-scaled
+// FP4 MMAs on operands resident in shared memory, with nothing else in the
+// loop, so the elapsed time measures the instruction rate the tensor cores
+// sustain on this part (the denominator the GEMM's tensor-pipe fraction is
+// reported against, next to the nominal figure).  Variants:
+//   0  cta_group::1, kind::mxf4nvf4 (NVFP4 scales), 128 x 256 x 64 per MMA
+//   1  as 0, plus the 3 scale-factor copies (tcgen05.cp) per MMA that a GEMM
+//      K step needs
+//   2  cta_group::2, 256 x 256 x 64 per MMA (CTA pair)
+//   3  as 2, plus the scale-factor copies
+// Operands are filled with pseudo-random codes and unit scales.  Waits are
+// bounded like the GEMM's.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "internal.h"
+#include "sm100_ptx.cuh"
+
+namespace fp4impl {
+namespace {
+using namespace ptx;
+
+constexpr int A_BYTES = 128 * 128;      // 128 rows x 256 FP4
+constexpr int B_BYTES = 256 * 128;      // 256 rows (1 SM) / 128 rows per CTA (pair)
+constexpr int SF_BYTES = 3 * 512;
+constexpr int PEAK_SMEM = A_BYTES + B_BYTES + SF_BYTES + 1024 + 64;
+
+__device__ __forceinline__ uint32_t hash32(uint32_t x) {
+  x ^= x >> 16; x *= 0x7FEB352Du; x ^= x >> 15; x *= 0x846CA68Bu; x ^= x >> 16;
+  return x;
+}
+
+template <bool PAIR, bool WITH_CP>
+__device__ void peak_body(int iters, uint32_t* status, uint8_t* base) {
+  uint8_t* sA = base;
+  uint8_t* sB = base + A_BYTES;
+  uint8_t* sSF = base + A_BYTES + B_BYTES;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sSF + SF_BYTES);
+  uint32_t* holder = reinterpret_cast<uint32_t*>(bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
+  const int t = threadIdx.x;
+  // random E2M1 codes (no NaN in FP4), unit E4M3 scales (0x38 = 1.0)
+  for (int i = t; i < (A_BYTES + B_BYTES) / 4; i += blockDim.x)
+    reinterpret_cast<uint32_t*>(sA)[i] = hash32(i * 2654435761u + blockIdx.x);
+  for (int i = t; i < SF_BYTES; i += blockDim.x) sSF[i] = 0x38;
+  if (t == 0) {
+    mbar_init(smem_u32(bar), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  if (t < 32) {
+    if (PAIR) tmem_alloc_pair(smem_u32(holder), 512);
+    else tmem_alloc(smem_u32(holder), 512);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (PAIR) cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = *holder;
+  const bool issuer = PAIR ? (cluster_ctarank() == 0 && t == 0) : (t == 0);
+  if (issuer) {
+    const uint32_t t_sfa = tmem + 256, t_sfb = tmem + 260;
+    const uint64_t sf0 = smem_desc(smem_u32(sSF), 0, 128, 0);
+    const uint64_t sf1 = smem_desc(smem_u32(sSF + 512), 0, 128, 0);
+    const uint64_t sf2 = smem_desc(smem_u32(sSF + 1024), 0, 128, 0);
+    auto cp_all = [&]() {
+      if (PAIR) {
+        tc_cp_pair_32x128b(t_sfa, sf0); tc_cp_pair_32x128b(t_sfb, sf1); tc_cp_pair_32x128b(t_sfb + 4, sf2);
+      } else {
+        tc_cp_32x128b(t_sfa, sf0); tc_cp_32x128b(t_sfb, sf1); tc_cp_32x128b(t_sfb + 4, sf2);
+      }
+    };
+    cp_all();
+    const uint32_t idesc = make_idesc(256, PAIR ? 256 : 128, 0u, 0u, 0u);
+    const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
+    for (int i = 0; i < iters; ++i) {
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        if (WITH_CP) cp_all();
+        const uint64_t ad = smem_desc(a_base + kk * 32, 16, 1024, 2);
+        const uint64_t bd = smem_desc(b_base + kk * 32, 16, 1024, 2);
+        if (PAIR) tc_mma_pair<true>(tmem, ad, bd, idesc, t_sfa, t_sfb, 1u);
+        else tc_mma<true>(tmem, ad, bd, idesc, t_sfa, t_sfb, 1u);
+      }
+    }
+    if (PAIR) tc_commit_pair(smem_u32(bar), 0x1);
+    else tc_commit(smem_u32(bar));
+    mbar_wait(smem_u32(bar), 0, abort_flag, status, 0x2000);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (PAIR) cluster_sync();
+  if (t < 32) {
+    tc_fence_after();
+    if (PAIR) tmem_dealloc_pair(tmem, 512);
+    else tmem_dealloc(tmem, 512);
+  }
+}
+
+template <bool WITH_CP>
+__global__ void __launch_bounds__(128, 1) mma_peak_single(int iters, uint32_t* status) {
+  extern __shared__ uint8_t sm[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm) + 1023) & ~uintptr_t(1023));
+  peak_body<false, WITH_CP>(iters, status, base);
+}
+
+template <bool WITH_CP>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1)
+mma_peak_pair(int iters, uint32_t* status) {
+  extern __shared__ uint8_t sm[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm) + 1023) & ~uintptr_t(1023));
+  peak_body<true, WITH_CP>(iters, status, base);
+}
+
+}  // namespace
+}  // namespace fp4impl
+
+using namespace fp4impl;
+
+extern "C" fp4_status fp4_mma_rate(int32_t variant, int32_t iters, float* tflops_out,
+                                   void* ws, size_t ws_bytes, void* stream) {
+  if (tflops_out == nullptr || ws == nullptr) return FP4_ERR_NULL;
+  if (ws_bytes < sizeof(DeviceStatus)) return FP4_ERR_WORKSPACE;
+  if (variant < 0 || variant > 3 || iters <= 0) return FP4_ERR_SHAPE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int grid = (sm_count() / 2) * 2;
+  uint32_t* status = static_cast<uint32_t*>(ws);
+  cudaEvent_t e0, e1;
+  if (cudaEventCreate(&e0) != cudaSuccess || cudaEventCreate(&e1) != cudaSuccess) return FP4_ERR_CUDA;
+  auto launch = [&]() {
+    switch (variant) {
+      case 0: cudaFuncSetAttribute(mma_peak_single<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, PEAK_SMEM);
+              mma_peak_single<false><<<grid, 128, PEAK_SMEM, s>>>(iters, status); break;
+      case 1: cudaFuncSetAttribute(mma_peak_single<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, PEAK_SMEM);
+              mma_peak_single<true><<<grid, 128, PEAK_SMEM, s>>>(iters, status); break;
+      case 2: cudaFuncSetAttribute(mma_peak_pair<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, PEAK_SMEM);
+              mma_peak_pair<false><<<grid, 128, PEAK_SMEM, s>>>(iters, status); break;
+      default: cudaFuncSetAttribute(mma_peak_pair<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, PEAK_SMEM);
+               mma_peak_pair<true><<<grid, 128, PEAK_SMEM, s>>>(iters, status); break;
+    }
+    count_launches(1);
+  };
+  launch();                                   // warm-up
+  cudaEventRecord(e0, s);
+  launch();
+  cudaEventRecord(e1, s);
+  fp4_status st = FP4_OK;
+  if (cudaEventSynchronize(e1) != cudaSuccess || cudaGetLastError() != cudaSuccess) st = FP4_ERR_CUDA;
+  float ms = 0.0f;
+  cudaEventElapsedTime(&ms, e0, e1);
+  cudaEventDestroy(e0);
+  cudaEventDestroy(e1);
+  // flops: each CTA (single) or CTA pair issues iters * 4 MMAs of
+  // 128x256x64 (single) or 256x256x64 (pair)
+  const double per_mma = (variant < 2) ? 2.0 * 128 * 256 * 64 : 2.0 * 256 * 256 * 64;
+  const double issuers = (variant < 2) ? grid : grid / 2;
+  *tflops_out = (float)(issuers * 4.0 * iters * per_mma / (ms * 1e-3) / 1e12);
+  return st;
+}

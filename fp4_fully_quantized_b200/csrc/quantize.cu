@@ -105,6 +105,47 @@ amax_rows_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols
   block_amax_atomic(m, amax);
 }
 
+// Plain amax (no rotation): 4 independent 16-byte loads per thread in
+// flight; |x| max taken on the BF16 bit patterns two at a time (sign bits
+// cleared, per-halfword unsigned max), which is exact and keeps NaN
+// patterns above +Inf.
+__global__ void __launch_bounds__(kThreads)
+amax_plain_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+                  float* amax) {
+  const int64_t cpr = cols >> 3;
+  const int64_t total = rows * cpr;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  uint32_t m2 = 0;
+  const bool dense = (ld == cols);
+  int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  for (; g + 3 * stride < total; g += 4 * stride) {
+    uint4 u[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int64_t gg = g + q * stride;
+      const int64_t off = dense ? gg * 8 : (gg / cpr) * ld + (gg % cpr) * 8;
+      u[q] = ld_nc_v4(x + off);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      m2 = __vmaxu2(m2, u[q].x & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, u[q].y & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, u[q].z & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, u[q].w & 0x7FFF7FFFu);
+    }
+  }
+  for (; g < total; g += stride) {
+    const int64_t off = dense ? g * 8 : (g / cpr) * ld + (g % cpr) * 8;
+    const uint4 u = ld_nc_v4(x + off);
+    m2 = __vmaxu2(m2, u.x & 0x7FFF7FFFu);
+    m2 = __vmaxu2(m2, u.y & 0x7FFF7FFFu);
+    m2 = __vmaxu2(m2, u.z & 0x7FFF7FFFu);
+    m2 = __vmaxu2(m2, u.w & 0x7FFF7FFFu);
+  }
+  const uint32_t hi = m2 >> 16, lo = m2 & 0xFFFFu;
+  block_amax_atomic(__uint_as_float(max(hi, lo) << 16), amax);
+}
+
 // ---------------------------------------------------------------------------
 // Row-wise quantization (NVFP4 BS = 16 or MXFP4 BS = 32).
 // ---------------------------------------------------------------------------
@@ -439,6 +480,225 @@ quant_2d_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols,
   }
 }
 
+// ---------------------------------------------------------------------------
+// Fused row-wise + transposed quantization: each 64 x 256 tile of x is read
+// from HBM once (cp.async into a double-buffered shared tile, the next tile in
+// flight while this one is encoded) and produces both outputs:
+//   row phase   warp w takes rows w, w + 8, ...; lane l the 8 values at columns
+//               8l .. 8l + 7 (blocks of 16/32 = 2/4 adjacent lanes, Hadamard
+//               stages across lanes by shuffles), 4 code bytes per lane;
+//   column phase thread t takes column t, rows in two runs of 32 (blocks run
+//               down the column), 16 code bytes per run of the transposed
+//               operand.
+// ---------------------------------------------------------------------------
+constexpr int kDualTM = 64, kDualTK = 256, kDualThreads = 256;
+constexpr int kDualSmem = 2 * kDualTM * kDualTK * 2;   // two bf16 tiles: 64 KB
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, bool valid) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  const int n = valid ? 16 : 0;                        // 0 source bytes: zero fill
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(gsrc), "r"(n)
+               : "memory");
+}
+
+template <bool NV>
+__device__ __forceinline__ void block_scale(float bmax, float s_enc, const float* inv_tab,
+                                            uint32_t& sf, float& inv) {
+  if constexpr (NV) {
+    const float t = __fdiv_rn(__fmul_rn(bmax, s_enc), 6.0f);
+    sf = e4m3_rn_sat(t);                  // 0 .. 126 (satfinite)
+    inv = inv_tab[sf];                    // RN(s_enc / value(sf)), 0 for sf = 0
+  } else {
+    int e = (bmax == 0.0f) ? -127 : floor_log2_f32(bmax) - 2;
+    e = max(-127, min(127, e));
+    sf = (uint32_t)(e + 127);
+    inv = exp2_neg_exact(e);
+  }
+}
+
+template <int BS, int RHT_R, int RHT_C, bool SR_R, bool SR_C>
+__global__ void __launch_bounds__(kDualThreads, 2)
+quant_dual_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+                  uint32_t mask_r, uint32_t mask_c, uint64_t sr_seed, uint32_t stream_r,
+                  uint32_t stream_c, const float* __restrict__ amax_src_r,
+                  const float* __restrict__ amax_src_c, float* amax_out_r, float* amax_out_c,
+                  float* s_dec_r, float* s_dec_c, uint8_t* __restrict__ codes_r,
+                  uint8_t* __restrict__ scales_r, uint8_t* __restrict__ mma_r,
+                  uint8_t* __restrict__ codes_c, uint8_t* __restrict__ scales_c,
+                  uint8_t* __restrict__ mma_c, uint32_t* status) {
+  constexpr bool NV = (BS == 16);
+  constexpr int TPB = BS / 8;
+  extern __shared__ __align__(16) uint8_t dual_smem[];
+  __nv_bfloat16 (*tile)[kDualTM][kDualTK] =
+      reinterpret_cast<__nv_bfloat16 (*)[kDualTM][kDualTK]>(dual_smem);
+
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int64_t tiles_k = (cols + kDualTK - 1) / kDualTK;
+  const int64_t ntiles = ((rows + kDualTM - 1) / kDualTM) * tiles_k;
+  const int64_t S_r = cols / BS, S_r4 = (S_r + 3) & ~3LL;   // blocks per row, row output
+  const int64_t S_c = rows / BS, S_c4 = (S_c + 3) & ~3LL;   // blocks per row of x^T
+
+  float se_r = 1.0f, sd_r = 1.0f, se_c = 1.0f, sd_c = 1.0f;
+  if constexpr (NV) {
+    const float Ar = *amax_src_r, Ac = *amax_src_c;
+    if ((!(Ar <= FLT_MAX) || !(Ac <= FLT_MAX)) && blockIdx.x == 0 && t == 0)
+      set_status(status, FP4_ERR_NONFINITE, 4);
+    nvfp4_global_scales(Ar, se_r, sd_r);
+    nvfp4_global_scales(Ac, se_c, sd_c);
+    if (blockIdx.x == 0 && t == 0) {
+      if (amax_out_r != amax_src_r) *amax_out_r = Ar;
+      if (amax_out_c != amax_src_c) *amax_out_c = Ac;
+    }
+  }
+  if (blockIdx.x == 0 && t == 0) { *s_dec_r = sd_r; *s_dec_c = sd_c; }
+  // RN(s_enc / value(sf)) for every E4M3 code, both orientations (NVFP4);
+  // the first tile's __syncthreads publishes it.
+  __shared__ float inv_tab[2][128];
+  if constexpr (NV) {
+    const int o = t >> 7, code = t & 127;
+    const float se = o ? se_c : se_r;
+    inv_tab[o][code] = (code == 0 || code == 127)
+                           ? 0.0f : fminf(__fdiv_rn(se, e4m3_value((uint32_t)code)), FLT_MAX);
+  }
+  PhiloxKeys K;
+  if constexpr (SR_R || SR_C) K = philox_keys(sr_seed);
+
+  auto issue = [&](int64_t tile_id, int buf) {
+    const int64_t m0 = (tile_id / tiles_k) * kDualTM, k0 = (tile_id % tiles_k) * kDualTK;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int rr = i * 8 + warp, cc = lane * 8;
+      const bool ok = (m0 + rr < rows) && (k0 + cc < cols);
+      const __nv_bfloat16* src = ok ? x + (m0 + rr) * ld + k0 + cc : x;
+      cp_async16(&tile[buf][rr][cc], src, ok);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+
+  int64_t tile_id = blockIdx.x;
+  if (tile_id < ntiles) issue(tile_id, 0);
+  for (int it = 0; tile_id < ntiles; tile_id += gridDim.x, ++it) {
+    const int buf = it & 1;
+    const int64_t next = tile_id + gridDim.x;
+    if (next < ntiles) {
+      issue(next, buf ^ 1);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
+    __syncthreads();
+    const int64_t m0 = (tile_id / tiles_k) * kDualTM, k0 = (tile_id % tiles_k) * kDualTK;
+
+    // ---------------- row phase (blocks along x's rows) -----------------
+#pragma unroll 2
+    for (int i = 0; i < 8; ++i) {
+      const int rr = i * 8 + warp, cc = lane * 8;
+      const int64_t r = m0 + rr, c = k0 + cc;
+      const bool active = (r < rows) && (c < cols);
+      float v[8];
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(&tile[buf][rr][cc]), v);
+      if constexpr (RHT_R > 0) rht_chunk<RHT_R>(v, mask_r, lane % (RHT_R / 8));
+      float bmax = 0.0f;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) bmax = fmaxf(bmax, fabsf(v[q]));
+#pragma unroll
+      for (int lx = 1; lx < TPB; lx <<= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xFFFFFFFFu, bmax, lx));
+      uint32_t sf;
+      float inv;
+      block_scale<NV>(bmax, se_r, inv_tab[0], sf, inv);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = __fmul_rn(v[q], inv);
+      uint32_t packed;
+      if constexpr (!SR_R) {
+        packed = e2m1x8_rn(v);
+      } else {
+        const uint64_t i0 = (uint64_t)r * (uint64_t)cols + (uint64_t)c;
+        const U4 w0 = philox_keyed(i0 >> 2, stream_r, K);
+        const U4 w1 = philox_keyed((i0 >> 2) + 1, stream_r, K);
+        const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        packed = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) packed |= e2m1_sr_bits(v[q], u[q]) << (4 * q);
+      }
+      if (active) {
+        *reinterpret_cast<uint32_t*>(codes_r + r * (cols >> 1) + (c >> 1)) = packed;
+        if ((lane % TPB) == 0) {
+          const int64_t sb = c / BS;
+          if (scales_r != nullptr) scales_r[r * S_r + sb] = (uint8_t)sf;
+          if (mma_r != nullptr) mma_r[mma_sf_offset(r, sb, S_r4)] = (uint8_t)sf;
+        }
+      }
+    }
+
+    // ---------------- column phase (blocks along x's columns) -----------
+    const int64_t k = k0 + t;
+#pragma unroll 1
+    for (int h = 0; h < 2; ++h) {
+      const int64_t mrow0 = m0 + 32 * h;
+      if (k >= cols || mrow0 >= rows) continue;
+      float v[32];
+#pragma unroll
+      for (int q = 0; q < 32; ++q) v[q] = __bfloat162float(tile[buf][32 * h + q][t]);
+      if constexpr (RHT_C > 0) {
+#pragma unroll
+        for (int base = 0; base < 32; base += RHT_C) {
+#pragma unroll
+          for (int q = 0; q < RHT_C; ++q)
+            if ((mask_c >> q) & 1u) v[base + q] = -v[base + q];
+#pragma unroll
+          for (int hh = 1; hh < RHT_C; hh <<= 1) {
+#pragma unroll
+            for (int q = 0; q < RHT_C; ++q) {
+              if (q & hh) continue;
+              const float a = v[base + q], b = v[base + q + hh];
+              v[base + q] = __fadd_rn(a, b);
+              v[base + q + hh] = __fsub_rn(a, b);
+            }
+          }
+          const float cn = rht_scale<RHT_C>();
+#pragma unroll
+          for (int q = 0; q < RHT_C; ++q) v[base + q] = __fmul_rn(v[base + q], cn);
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < 32 / BS; ++b) {
+        float bmax = 0.0f;
+#pragma unroll
+        for (int q = 0; q < BS; ++q) bmax = fmaxf(bmax, fabsf(v[b * BS + q]));
+        uint32_t sf;
+        float inv;
+        block_scale<NV>(bmax, se_c, inv_tab[1], sf, inv);
+#pragma unroll
+        for (int q = 0; q < BS; ++q) v[b * BS + q] = __fmul_rn(v[b * BS + q], inv);
+        if (mrow0 + b * BS < rows) {
+          const int64_t sb = (mrow0 + b * BS) / BS;
+          if (scales_c != nullptr) scales_c[k * S_c + sb] = (uint8_t)sf;
+          if (mma_c != nullptr) mma_c[mma_sf_offset(k, sb, S_c4)] = (uint8_t)sf;
+        }
+      }
+      uint32_t packed[4] = {0, 0, 0, 0};
+      if constexpr (!SR_C) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) packed[q] = e2m1x8_rn(&v[8 * q]);
+      } else {
+        const uint64_t i0 = (uint64_t)k * (uint64_t)rows + (uint64_t)mrow0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const U4 w = philox_keyed((i0 >> 2) + q, stream_c, K);
+          const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            packed[q >> 1] |= e2m1_sr_bits(v[4 * q + e], u[e]) << (4 * ((4 * q + e) & 7));
+        }
+      }
+      uint8_t* dst = codes_c + k * (rows >> 1) + (mrow0 >> 1);
+      *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+      if (mrow0 + 16 < rows) *reinterpret_cast<uint2*>(dst + 8) = make_uint2(packed[2], packed[3]);
+    }
+    __syncthreads();          // all reads of this buffer done before it is refilled
+  }
+}
+
 int grid_for(int64_t work_items, int per_block, int max_blocks_per_sm) {
   int64_t need = (work_items + per_block - 1) / per_block;
   const int64_t cap = (int64_t)sm_count() * max_blocks_per_sm;
@@ -454,8 +714,14 @@ int grid_for(int64_t work_items, int per_block, int max_blocks_per_sm) {
 // ---------------------------------------------------------------------------
 cudaError_t launch_amax_rows(const void* x, int64_t rows, int64_t cols, int64_t ld, int rht_n,
                              uint32_t mask, float* amax, cudaStream_t s) {
-  const int grid = grid_for(rows * (cols / 8), kThreads, 8);
   auto xp = static_cast<const __nv_bfloat16*>(x);
+  if (rht_n == 0) {
+    const int g = grid_for(rows * (cols / 8), kThreads * 4, 8);
+    amax_plain_kernel<<<g, kThreads, 0, s>>>(xp, rows, cols, ld, amax);
+    count_launches(1);
+    return cudaGetLastError();
+  }
+  const int grid = grid_for(rows * (cols / 8), kThreads, 8);
   if (rht_n == 16) amax_rows_kernel<16><<<grid, kThreads, 0, s>>>(xp, rows, cols, ld, mask, amax);
   else if (rht_n == 32) amax_rows_kernel<32><<<grid, kThreads, 0, s>>>(xp, rows, cols, ld, mask, amax);
   else amax_rows_kernel<0><<<grid, kThreads, 0, s>>>(xp, rows, cols, ld, mask, amax);
@@ -519,6 +785,43 @@ cudaError_t launch_quant_cols(const RowQuantArgs& a, cudaStream_t s) {
   FP4_DISPATCH(cols_variant, a, grid, s);
   count_launches(1);
   return cudaGetLastError();
+}
+
+template <int BS, int RR, int RC, bool SRR, bool SRC>
+static cudaError_t dual_variant(const DualQuantArgs& a, cudaStream_t s) {
+  auto kern = quant_dual_kernel<BS, RR, RC, SRR, SRC>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDualSmem);
+  if (e != cudaSuccess) return e;
+  const int64_t ntiles = ((a.rows + kDualTM - 1) / kDualTM) * ((a.cols + kDualTK - 1) / kDualTK);
+  const int grid = grid_for(ntiles, 1, 2);
+  kern<<<grid, kDualThreads, kDualSmem, s>>>(
+      static_cast<const __nv_bfloat16*>(a.x), a.rows, a.cols, a.ld, a.mask_r, a.mask_c, a.sr_seed,
+      a.stream_r, a.stream_c, a.amax_src_r, a.amax_src_c, a.amax_out_r, a.amax_out_c, a.s_dec_r,
+      a.s_dec_c, a.codes_r, a.scales_r, a.mma_r, a.codes_c, a.scales_c, a.mma_c, a.status);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+template <int BS, int RR, int RC>
+static cudaError_t dual_rounding(const DualQuantArgs& a, cudaStream_t s) {
+  if (a.sr_r) return a.sr_c ? dual_variant<BS, RR, RC, true, true>(a, s)
+                            : dual_variant<BS, RR, RC, true, false>(a, s);
+  return a.sr_c ? dual_variant<BS, RR, RC, false, true>(a, s)
+                : dual_variant<BS, RR, RC, false, false>(a, s);
+}
+
+bool dual_supported(int fmt, int rht_r, int rht_c) {
+  const int n = fmt == FP4_NVFP4 ? 16 : 32;
+  return (rht_r == 0 || rht_r == n) && (rht_c == 0 || rht_c == n);
+}
+
+cudaError_t launch_quant_dual(const DualQuantArgs& a, cudaStream_t s) {
+  if (a.fmt == FP4_NVFP4) {
+    if (a.rht_r) return a.rht_c ? dual_rounding<16, 16, 16>(a, s) : dual_rounding<16, 16, 0>(a, s);
+    return a.rht_c ? dual_rounding<16, 0, 16>(a, s) : dual_rounding<16, 0, 0>(a, s);
+  }
+  if (a.rht_r) return a.rht_c ? dual_rounding<32, 32, 32>(a, s) : dual_rounding<32, 32, 0>(a, s);
+  return a.rht_c ? dual_rounding<32, 0, 32>(a, s) : dual_rounding<32, 0, 0>(a, s);
 }
 
 cudaError_t launch_quant_2d(const Quant2DArgs& a, cudaStream_t s) {

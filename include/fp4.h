@@ -149,7 +149,8 @@ void fp4_qparams_default(fp4_qparams* p);
 size_t fp4_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* Quantize x (BF16, [rows, cols] with leading dimension ld >= cols, in
- * elements, ld % 8 == 0) into `out` (row-wise, may be NULL) and/or `out_t`
+ * elements, ld % 8 == 0; NULL allowed when rows or cols is 0, which only
+ * writes amax = 0 and s_dec = 1) into `out` (row-wise, may be NULL) and/or `out_t`
  * (transposed, may be NULL).  Shape rules: NVFP4 1-D needs cols % 16 == 0
  * for `out` and rows % 16 == 0 for `out_t`; MXFP4 the same with 32; NVFP4
  * 2-D needs rows % 16 == 0 and cols % 16 == 0 and produces W (`out`) and
@@ -255,6 +256,17 @@ fp4_status fp4_clear_device_status(void* ws, void* stream);
 
 const char* fp4_status_str(int32_t status);
 int32_t fp4_abi_version(void);
+
+/* Tensor-core rate microbenchmark (synchronises `stream`): one persistent CTA
+ * (variants 0, 1) or CTA pair (2, 3) per SM issues `iters` x 4 back-to-back
+ * block-scaled NVFP4 MMAs (128x256x64, or 256x256x64 for a pair) on operands
+ * resident in shared memory; variants 1 and 3 add the three scale-factor
+ * copies into tensor memory that one MMA of a GEMM K step needs.  Writes the
+ * achieved TFLOP/s.  The measured rate is the denominator the GEMM's
+ * tensor-pipe fraction is reported against ("FP4" page, Hardware: FP4 on
+ * fifth-generation Tensor Cores). */
+fp4_status fp4_mma_rate(int32_t variant, int32_t iters, float* tflops_out, void* ws,
+                        size_t ws_bytes, void* stream);
 
 /* Number of CUDA kernels this library has enqueued in the calling process
  * since it was loaded (all devices, all streams).  Host-side counter, no
