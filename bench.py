@@ -367,7 +367,7 @@ def run_ours(args, rank, world, device):
                    else "RTN fwd/bwd", "weights": "16x16 tiles" if fmt == F.NVFP4 else "1x32",
                    "rht": {0: "off", 4: "wgrad 16-pt", 7: "all GEMMs 32-pt"}.get(cfg.rht_mask),
                    "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}"},
-        "roofline": {"kernel": "fp4_gemm_kernel (tcgen05 block-scaled)", "bound": "tensor",
+        "roofline": {"kernel": "fp4_gemm_sfst_kernel (tcgen05 block-scaled, scales staged by tcgen05.st)", "bound": "tensor",
                      "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1),
                      "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4),
                      "peak_source": f"{pk_src}: bf16 sustained x {FP4_PER_BF16:g} (nominal FP4/BF16)",
@@ -415,7 +415,8 @@ def run_reference(args):
 def run_case(args, device):
     """A single kernel family on one small problem (for profiler captures):
     --case gemm: NVFP4 fprop-style GEMM [m, k] x [n, k]^T, BF16 out;
-    --case quant: NVFP4 row-wise RTN + transposed SR of a [m, k] tensor."""
+    --case quant: NVFP4 row-wise RTN + transposed SR of a [m, k] tensor;
+    --case quant_sr: both outputs stochastically rounded (the dY quantization)."""
     import fp4_fully_quantized_b200 as F
     import fqt_synth as S
     F.load()
@@ -424,9 +425,10 @@ def run_case(args, device):
     x = S.student_t_channels(M, K, seed=1)[0].to(device)
     qa = F.QTensor.empty(M, K, device=device, logical_scales=False)
     qat = F.QTensor.empty(K, M, device=device, logical_scales=False)
-    if args.case == "quant":
-        fn = lambda: F.fp4_quantize(x, qa, qat, round=F.RTN, round_t=F.SR, sr_seed=1, sr_stream_t=3,
-                                    ws=ws)
+    if args.case in ("quant", "quant_sr"):
+        r = F.SR if args.case == "quant_sr" else F.RTN
+        fn = lambda: F.fp4_quantize(x, qa, qat, round=r, round_t=F.SR, sr_seed=1, sr_stream=1,
+                                    sr_stream_t=3, ws=ws)
         units, unit = M * K * Q_BYTES_PER_ELEM / 1e9, "GB/s"
     else:
         w = S.normal((N, K), 0.02, seed=2).to(device)
@@ -454,7 +456,7 @@ def run_case(args, device):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--case", choices=["gemm", "quant"], default=None,
+    ap.add_argument("--case", choices=["gemm", "quant", "quant_sr"], default=None,
                     help="time one kernel family on a small problem (profiling)")
     ap.add_argument("--m", type=int, default=8192)
     ap.add_argument("--n", type=int, default=4096)

@@ -492,6 +492,10 @@ quant_2d_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols,
 //               operand.
 // ---------------------------------------------------------------------------
 constexpr int kDualTM = 64, kDualTK = 256, kDualThreads = 256;
+#ifndef FP4_DUAL_CTAS_PER_SM
+#define FP4_DUAL_CTAS_PER_SM 3
+#endif
+constexpr int kDualCtasPerSm = FP4_DUAL_CTAS_PER_SM;   // resident CTAs per SM
 constexpr int kDualSmem = 2 * kDualTM * kDualTK * 2;   // two bf16 tiles: 64 KB
 
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, bool valid) {
@@ -517,7 +521,7 @@ __device__ __forceinline__ void block_scale(float bmax, float s_enc, const float
 }
 
 template <int BS, int RHT_R, int RHT_C, bool SR_R, bool SR_C>
-__global__ void __launch_bounds__(kDualThreads, 2)
+__global__ void __launch_bounds__(kDualThreads, kDualCtasPerSm)
 quant_dual_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
                   uint32_t mask_r, uint32_t mask_c, uint64_t sr_seed, uint32_t stream_r,
                   uint32_t stream_c, const float* __restrict__ amax_src_r,
@@ -793,7 +797,7 @@ static cudaError_t dual_variant(const DualQuantArgs& a, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDualSmem);
   if (e != cudaSuccess) return e;
   const int64_t ntiles = ((a.rows + kDualTM - 1) / kDualTM) * ((a.cols + kDualTK - 1) / kDualTK);
-  const int grid = grid_for(ntiles, 1, 2);
+  const int grid = grid_for(ntiles, 1, kDualCtasPerSm);
   kern<<<grid, kDualThreads, kDualSmem, s>>>(
       static_cast<const __nv_bfloat16*>(a.x), a.rows, a.cols, a.ld, a.mask_r, a.mask_c, a.sr_seed,
       a.stream_r, a.stream_c, a.amax_src_r, a.amax_src_c, a.amax_out_r, a.amax_out_c, a.s_dec_r,
