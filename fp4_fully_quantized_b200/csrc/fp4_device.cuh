@@ -131,52 +131,26 @@ __device__ __forceinline__ uint32_t e2m1x8_rn(const float* v) {
 
 // E2M1 stochastic rounding of one value with draw u: with lo <= |v| <= hi the
 // neighbouring levels (|v| clamped to 6), round up iff u < ceil(p * 2^32),
-// p = (|v| - lo) / (hi - lo).  Level gaps: 0.5 below 2, 1 in [2, 4), 2 in
-// [4, 6].  Returns the 4-bit code (sign kept, also for results of 0).
+// p = (|v| - lo) / (hi - lo).  Returns the 4-bit code (sign kept, also for
+// results of 0).
+//
+// Branch-free and mostly off the integer ALU pipe.  For |v| >= 1 the grid
+// splits each binade of binary32 in two (gaps 0.5, 1, 2), so the lower level
+// is (exponent, top mantissa bit) = bits >> 22, less 252, and ceil(p * 2^32)
+// is the remaining 22 mantissa bits, i.e. bits << 10.  For |v| < 1 the gap
+// is 0.5 everywhere: with Y = |v| * 2^33 (exact), the lower level is 1 iff
+// Y >= 2^32 and p * 2^32 = Y mod 2^32 (exact), rounded up to an integer.
 __device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t u) {
-  const uint32_t sign = (__float_as_uint(v) >> 31) << 3;
-  float a = fminf(fabsf(v), 6.0f);
-  float gap_scale, lo;           // gap_scale = 2^32 / gap
-  uint32_t code_lo;
-  if (a < 2.0f) {
-    float f = floorf(__fmul_rn(a, 2.0f));
-    lo = __fmul_rn(f, 0.5f);
-    code_lo = (uint32_t)f;
-    gap_scale = 8589934592.0f;   // 2^33
-  } else if (a < 4.0f) {
-    float f = floorf(a);
-    lo = f;
-    code_lo = (uint32_t)f + 2u;
-    gap_scale = 4294967296.0f;   // 2^32
-  } else {
-    lo = (a < 6.0f) ? 4.0f : 6.0f;
-    code_lo = (a < 6.0f) ? 6u : 7u;
-    gap_scale = 2147483648.0f;   // 2^31
-  }
-  const float y = __fmul_rn(__fsub_rn(a, lo), gap_scale);   // exact, < 2^32
-  const unsigned long long T = __float2ull_ru(y);            // ceil, exact
-  const uint32_t up = ((unsigned long long)u < T) ? 1u : 0u;
-  return sign | (code_lo + up);
-}
-
-// The same stochastic rounding read from the binary32 encoding of |v|
-// (clamped to 6), branch-free.  Within [1, 6] the E2M1 grid splits each
-// binade in two, so the level is (exponent, top mantissa bit) and the
-// fraction of the gap is the remaining 22 mantissa bits: ceil(p * 2^32) is
-// exactly those bits << 10.  In [0.5, 1) the gap is the whole binade (bits
-// << 9); below 0.5 the gap is [0, 0.5] and ceil(p * 2^32) = ceil(|v| * 2^33).
-__device__ __forceinline__ uint32_t e2m1_sr_bits(float v, uint32_t u) {
-  const uint32_t bits = __float_as_uint(v);
-  const uint32_t sign = (bits >> 28) & 8u;
-  const uint32_t a = min(bits & 0x7FFFFFFFu, 0x40C00000u);      // |v| clamped to 6.0
-  const uint32_t E = a >> 23, m = a & 0x7FFFFFu;
-  const uint32_t code_hi = ((E - 126u) << 1) | (m >> 22);        // a >= 1
-  const uint32_t t_hi = (m & 0x3FFFFFu) << 10;
-  const uint32_t t_mid = m << 9;                                 // 0.5 <= a < 1
-  const uint32_t t_lo = __float2uint_ru(__fmul_rn(__uint_as_float(a), 8589934592.0f));  // a < 0.5
-  const uint32_t code_lo = E >= 127u ? code_hi : (E == 126u ? 1u : 0u);
-  const uint32_t T = E >= 127u ? t_hi : (E == 126u ? t_mid : t_lo);
-  return sign | (code_lo + (u < T ? 1u : 0u));
+  const float a = fminf(fabsf(v), 6.0f);
+  const uint32_t ab = __float_as_uint(a);
+  const float Y = __fmul_rn(a, 8589934592.0f);                      // 2^33
+  const bool half = Y >= 4294967296.0f;                             // |v| >= 0.5
+  const uint32_t t_small = __float2uint_ru(half ? __fadd_rn(Y, -4294967296.0f) : Y);
+  const bool big = ab >= 0x3F800000u;                               // |v| >= 1
+  const uint32_t T = big ? (ab << 10) : t_small;
+  const uint32_t lo = big ? (ab >> 22) - 252u : (half ? 1u : 0u);
+  const uint32_t sign = __umulhi(__float_as_uint(v), 16u) & 8u;     // bit 31 -> bit 3
+  return (lo + (u < T ? 1u : 0u)) | sign;
 }
 
 // ---------------------------------------------------------------------------

@@ -622,7 +622,7 @@ quant_dual_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t col
         const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
         packed = 0;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) packed |= e2m1_sr_bits(v[q], u[q]) << (4 * q);
+        for (int q = 0; q < 8; ++q) packed |= e2m1_sr(v[q], u[q]) << (4 * q);
       }
       if (active) {
         *reinterpret_cast<uint32_t*>(codes_r + r * (cols >> 1) + (c >> 1)) = packed;
@@ -692,7 +692,7 @@ quant_dual_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t col
           const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            packed[q >> 1] |= e2m1_sr_bits(v[4 * q + e], u[e]) << (4 * ((4 * q + e) & 7));
+            packed[q >> 1] |= e2m1_sr(v[4 * q + e], u[e]) << (4 * ((4 * q + e) & 7));
         }
       }
       uint8_t* dst = codes_c + k * (rows >> 1) + (mrow0 >> 1);
