@@ -50,13 +50,14 @@ __host__ __device__ __forceinline__ U4 philox4x32_10(uint64_t ctr_lo64, uint32_t
   return U4{c0, c1, c2, c3};
 }
 
-// The same generator with its ten round keys precomputed once per thread and
-// each 32x32 product done as one widening multiply (hi and lo together).
+// The same generator with its ten round keys precomputed (on the host, passed
+// as a kernel parameter so they live in the constant bank, not in registers)
+// and each 32x32 product done as one widening multiply (hi and lo together).
 struct PhiloxKeys {
   uint32_t k0[10], k1[10];
 };
 
-__device__ __forceinline__ PhiloxKeys philox_keys(uint64_t seed) {
+__host__ __device__ __forceinline__ PhiloxKeys philox_keys(uint64_t seed) {
   PhiloxKeys K;
   uint32_t a = (uint32_t)seed, b = (uint32_t)(seed >> 32);
 #pragma unroll
@@ -134,23 +135,22 @@ __device__ __forceinline__ uint32_t e2m1x8_rn(const float* v) {
 // p = (|v| - lo) / (hi - lo).  Returns the 4-bit code (sign kept, also for
 // results of 0).
 //
-// Branch-free and mostly off the integer ALU pipe.  For |v| >= 1 the grid
-// splits each binade of binary32 in two (gaps 0.5, 1, 2), so the lower level
-// is (exponent, top mantissa bit) = bits >> 22, less 252, and ceil(p * 2^32)
-// is the remaining 22 mantissa bits, i.e. bits << 10.  For |v| < 1 the gap
-// is 0.5 everywhere: with Y = |v| * 2^33 (exact), the lower level is 1 iff
-// Y >= 2^32 and p * 2^32 = Y mod 2^32 (exact), rounded up to an integer.
+// Branch-free, with the level and the threshold computed together as the two
+// halves of one 64-bit integer (high word: lower level index, low word:
+// ceil(p * 2^32)).  For |v| >= 1 the grid splits each binade of binary32 in
+// two (gaps 0.5, 1, 2), so the lower level is (exponent, top mantissa bit) =
+// bits >> 22, less 252, and ceil(p * 2^32) is the remaining 22 mantissa bits,
+// bits << 10: both halves of bits * 2^10 - 252 * 2^32.  For |v| < 1 the gap is
+// 0.5 everywhere and ceil(|v| * 2^33) (exact: the product is a float below
+// 2^33) has the level (0 or 1) above bit 32 and ceil(p * 2^32) below it.
 __device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t u) {
   const float a = fminf(fabsf(v), 6.0f);
   const uint32_t ab = __float_as_uint(a);
-  const float Y = __fmul_rn(a, 8589934592.0f);                      // 2^33
-  const bool half = Y >= 4294967296.0f;                             // |v| >= 0.5
-  const uint32_t t_small = __float2uint_ru(half ? __fadd_rn(Y, -4294967296.0f) : Y);
-  const bool big = ab >= 0x3F800000u;                               // |v| >= 1
-  const uint32_t T = big ? (ab << 10) : t_small;
-  const uint32_t lo = big ? (ab >> 22) - 252u : (half ? 1u : 0u);
-  const uint32_t sign = __umulhi(__float_as_uint(v), 16u) & 8u;     // bit 31 -> bit 3
-  return (lo + (u < T ? 1u : 0u)) | sign;
+  const uint64_t w_big = (uint64_t)ab * 1024u + 0xFFFFFF0400000000ull;
+  const uint64_t w_small = __float2ull_ru(__fmul_rn(a, 8589934592.0f));   // 2^33
+  const uint64_t w = ab >= 0x3F800000u ? w_big : w_small;
+  const uint32_t level = (uint32_t)(w >> 32) + ((uint32_t)w > u ? 1u : 0u);
+  return level + ((__float_as_uint(v) >> 31) << 3);
 }
 
 // ---------------------------------------------------------------------------

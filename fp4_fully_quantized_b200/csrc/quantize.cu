@@ -487,9 +487,9 @@ quant_2d_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols,
 //   row phase   warp w takes rows w, w + 8, ...; lane l the 8 values at columns
 //               8l .. 8l + 7 (blocks of 16/32 = 2/4 adjacent lanes, Hadamard
 //               stages across lanes by shuffles), 4 code bytes per lane;
-//   column phase thread t takes column t, rows in two runs of 32 (blocks run
-//               down the column), 16 code bytes per run of the transposed
-//               operand.
+//   column phase thread t takes column t, the tile's 64 rows block by block
+//               down the column, and writes its 32 code bytes and 4 (2)
+//               scale bytes of the transposed operand in one go.
 // ---------------------------------------------------------------------------
 constexpr int kDualTM = 64, kDualTK = 256, kDualThreads = 256;
 #ifndef FP4_DUAL_CTAS_PER_SM
@@ -523,7 +523,8 @@ __device__ __forceinline__ void block_scale(float bmax, float s_enc, const float
 template <int BS, int RHT_R, int RHT_C, bool SR_R, bool SR_C>
 __global__ void __launch_bounds__(kDualThreads, kDualCtasPerSm)
 quant_dual_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
-                  uint32_t mask_r, uint32_t mask_c, uint64_t sr_seed, uint32_t stream_r,
+                  uint32_t mask_r, uint32_t mask_c, const __grid_constant__ PhiloxKeys K,
+                  uint32_t stream_r,
                   uint32_t stream_c, const float* __restrict__ amax_src_r,
                   const float* __restrict__ amax_src_c, float* amax_out_r, float* amax_out_c,
                   float* s_dec_r, float* s_dec_c, uint8_t* __restrict__ codes_r,
@@ -564,8 +565,6 @@ quant_dual_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t col
     inv_tab[o][code] = (code == 0 || code == 127)
                            ? 0.0f : fminf(__fdiv_rn(se, e4m3_value((uint32_t)code)), FLT_MAX);
   }
-  PhiloxKeys K;
-  if constexpr (SR_R || SR_C) K = philox_keys(sr_seed);
 
   auto issue = [&](int64_t tile_id, int buf) {
     const int64_t m0 = (tile_id / tiles_k) * kDualTM, k0 = (tile_id % tiles_k) * kDualTK;
@@ -635,69 +634,97 @@ quant_dual_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t col
     }
 
     // ---------------- column phase (blocks along x's columns) -----------
+    // Thread t encodes column k0 + t over the tile's 64 rows (64/BS blocks),
+    // keeps the 32 code bytes and the block scales in registers and writes
+    // each with as few stores as alignment allows.
     const int64_t k = k0 + t;
-#pragma unroll 1
-    for (int h = 0; h < 2; ++h) {
-      const int64_t mrow0 = m0 + 32 * h;
-      if (k >= cols || mrow0 >= rows) continue;
-      float v[32];
+    if (k < cols) {
+      constexpr int NB = kDualTM / BS;                 // blocks per column in a tile
+      uint32_t cw[kDualTM / 8];                        // packed codes, 8 per word
+      uint32_t sfw = 0;                                // scale byte of block b at 8b
 #pragma unroll
-      for (int q = 0; q < 32; ++q) v[q] = __bfloat162float(tile[buf][32 * h + q][t]);
-      if constexpr (RHT_C > 0) {
+      for (int b = 0; b < NB; ++b) {
+        const int64_t mrow0 = m0 + BS * b;
 #pragma unroll
-        for (int base = 0; base < 32; base += RHT_C) {
+        for (int w = 0; w < BS / 8; ++w) cw[b * (BS / 8) + w] = 0;
+        if (mrow0 >= rows) continue;
+        float v[BS];
+#pragma unroll
+        for (int q = 0; q < BS; ++q) v[q] = __bfloat162float(tile[buf][BS * b + q][t]);
+        if constexpr (RHT_C > 0) {
 #pragma unroll
           for (int q = 0; q < RHT_C; ++q)
-            if ((mask_c >> q) & 1u) v[base + q] = -v[base + q];
+            if ((mask_c >> q) & 1u) v[q] = -v[q];
 #pragma unroll
           for (int hh = 1; hh < RHT_C; hh <<= 1) {
 #pragma unroll
             for (int q = 0; q < RHT_C; ++q) {
               if (q & hh) continue;
-              const float a = v[base + q], b = v[base + q + hh];
-              v[base + q] = __fadd_rn(a, b);
-              v[base + q + hh] = __fsub_rn(a, b);
+              const float x0 = v[q], x1 = v[q + hh];
+              v[q] = __fadd_rn(x0, x1);
+              v[q + hh] = __fsub_rn(x0, x1);
             }
           }
           const float cn = rht_scale<RHT_C>();
 #pragma unroll
-          for (int q = 0; q < RHT_C; ++q) v[base + q] = __fmul_rn(v[base + q], cn);
+          for (int q = 0; q < RHT_C; ++q) v[q] = __fmul_rn(v[q], cn);
         }
-      }
-#pragma unroll
-      for (int b = 0; b < 32 / BS; ++b) {
         float bmax = 0.0f;
 #pragma unroll
-        for (int q = 0; q < BS; ++q) bmax = fmaxf(bmax, fabsf(v[b * BS + q]));
+        for (int q = 0; q < BS; ++q) bmax = fmaxf(bmax, fabsf(v[q]));
         uint32_t sf;
         float inv;
         block_scale<NV>(bmax, se_c, inv_tab[1], sf, inv);
+        sfw |= sf << (8 * b);
 #pragma unroll
-        for (int q = 0; q < BS; ++q) v[b * BS + q] = __fmul_rn(v[b * BS + q], inv);
-        if (mrow0 + b * BS < rows) {
-          const int64_t sb = (mrow0 + b * BS) / BS;
-          if (scales_c != nullptr) scales_c[k * S_c + sb] = (uint8_t)sf;
-          if (mma_c != nullptr) mma_c[mma_sf_offset(k, sb, S_c4)] = (uint8_t)sf;
+        for (int q = 0; q < BS; ++q) v[q] = __fmul_rn(v[q], inv);
+        if constexpr (!SR_C) {
+#pragma unroll
+          for (int w = 0; w < BS / 8; ++w) cw[b * (BS / 8) + w] = e2m1x8_rn(&v[8 * w]);
+        } else {
+          const uint64_t i0 = (uint64_t)k * (uint64_t)rows + (uint64_t)mrow0;
+#pragma unroll
+          for (int q = 0; q < BS / 4; ++q) {
+            const U4 d = philox_keyed((i0 >> 2) + q, stream_c, K);
+            const uint32_t u[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              cw[b * (BS / 8) + (q >> 1)] += e2m1_sr(v[4 * q + e], u[e]) << (4 * ((4 * q + e) & 7));
+          }
         }
       }
-      uint32_t packed[4] = {0, 0, 0, 0};
-      if constexpr (!SR_C) {
+      const int64_t sb0 = m0 / BS;                     // first block of the tile
+      const int64_t left = (rows - m0) / BS;           // rows % BS == 0
+      const int nvalid = left < NB ? (int)left : NB;
+      uint8_t* dst = codes_c + k * (rows >> 1) + (m0 >> 1);
+      if (nvalid == NB && ((rows >> 1) & 15) == 0) {   // 16-byte aligned row of x^T
+        *reinterpret_cast<uint4*>(dst) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        *reinterpret_cast<uint4*>(dst + 16) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+      } else {                                         // rows % 16 == 0: 8-byte aligned
 #pragma unroll
-        for (int q = 0; q < 4; ++q) packed[q] = e2m1x8_rn(&v[8 * q]);
-      } else {
-        const uint64_t i0 = (uint64_t)k * (uint64_t)rows + (uint64_t)mrow0;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const U4 w = philox_keyed((i0 >> 2) + q, stream_c, K);
-          const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            packed[q >> 1] |= e2m1_sr(v[4 * q + e], u[e]) << (4 * ((4 * q + e) & 7));
+        for (int h = 0; h < kDualTM / 16; ++h)
+          if (16 * h < rows - m0) *reinterpret_cast<uint2*>(dst + 8 * h) = make_uint2(cw[2 * h], cw[2 * h + 1]);
+      }
+      if (scales_c != nullptr) {
+        uint8_t* sd = scales_c + k * S_c + sb0;
+        if (nvalid == NB && (S_c % NB) == 0 && (reinterpret_cast<uintptr_t>(scales_c) % NB) == 0) {
+          if constexpr (NB == 4) *reinterpret_cast<uint32_t*>(sd) = sfw;
+          else *reinterpret_cast<uint16_t*>(sd) = (uint16_t)sfw;
+        } else {
+          for (int b = 0; b < nvalid; ++b) sd[b] = (uint8_t)(sfw >> (8 * b));
         }
       }
-      uint8_t* dst = codes_c + k * (rows >> 1) + (mrow0 >> 1);
-      *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
-      if (mrow0 + 16 < rows) *reinterpret_cast<uint2*>(dst + 8) = make_uint2(packed[2], packed[3]);
+      if (mma_c != nullptr) {
+        // blocks sb0 .. sb0 + NB - 1 share one 4-byte slot group (sb0 % 4 == 0
+        // for NVFP4, sb0 % 2 == 0 for MXFP4): contiguous and aligned
+        uint8_t* md = mma_c + mma_sf_offset(k, sb0, S_c4);
+        if (nvalid == NB && (reinterpret_cast<uintptr_t>(mma_c) % NB) == 0) {
+          if constexpr (NB == 4) *reinterpret_cast<uint32_t*>(md) = sfw;
+          else *reinterpret_cast<uint16_t*>(md) = (uint16_t)sfw;
+        } else {
+          for (int b = 0; b < nvalid; ++b) md[b] = (uint8_t)(sfw >> (8 * b));
+        }
+      }
     }
     __syncthreads();          // all reads of this buffer done before it is refilled
   }
@@ -799,8 +826,9 @@ static cudaError_t dual_variant(const DualQuantArgs& a, cudaStream_t s) {
   const int64_t ntiles = ((a.rows + kDualTM - 1) / kDualTM) * ((a.cols + kDualTK - 1) / kDualTK);
   const int grid = grid_for(ntiles, 1, kDualCtasPerSm);
   kern<<<grid, kDualThreads, kDualSmem, s>>>(
-      static_cast<const __nv_bfloat16*>(a.x), a.rows, a.cols, a.ld, a.mask_r, a.mask_c, a.sr_seed,
-      a.stream_r, a.stream_c, a.amax_src_r, a.amax_src_c, a.amax_out_r, a.amax_out_c, a.s_dec_r,
+      static_cast<const __nv_bfloat16*>(a.x), a.rows, a.cols, a.ld, a.mask_r, a.mask_c,
+      philox_keys(a.sr_seed), a.stream_r, a.stream_c, a.amax_src_r, a.amax_src_c, a.amax_out_r,
+      a.amax_out_c, a.s_dec_r,
       a.s_dec_c, a.codes_r, a.scales_r, a.mma_r, a.codes_c, a.scales_c, a.mma_c, a.status);
   count_launches(1);
   return cudaGetLastError();
