@@ -264,6 +264,8 @@ fp4_gemm_sfst_kernel(const __grid_constant__ CUtensorMap tmap_a,
   } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + EPI_WARPS) {
     // ------------------------------------------------------------ epilogue
     const float scale = p.alpha * (*p.a_sdec) * (*p.b_sdec);
+    const int esize = p.out_f32 ? 4 : 2;
+    const bool wide_st = (reinterpret_cast<uintptr_t>(p.c) % 32) == 0 && (p.ldc * esize) % 32 == 0;
     float amax = 0.0f;
     uint32_t tile_iter = 0;
     const int quad = warp & 3, half = (warp - EPI_WARP0) >> 2;
@@ -297,9 +299,17 @@ fp4_gemm_sfst_kernel(const __grid_constant__ CUtensorMap tmap_a,
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_empty);
         if (ncols > 0) {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.c) + row * p.ldc + col);
+          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.c) + row * p.ldc + col;
+          if (wide_st) {          // full 32-byte sectors
 #pragma unroll
-          for (int q = 0; q < 16; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+            for (int q = 0; q < 8; ++q)
+              st_global_v8(dst + 16 * q, pk[8 * q], pk[8 * q + 1], pk[8 * q + 2], pk[8 * q + 3],
+                           pk[8 * q + 4], pk[8 * q + 5], pk[8 * q + 6], pk[8 * q + 7]);
+          } else {
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+            for (int q = 0; q < 16; ++q) d4[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          }
         }
       } else {
         // FP32: two halves of 64 columns; the accumulator is released after
@@ -318,14 +328,22 @@ fp4_gemm_sfst_kernel(const __grid_constant__ CUtensorMap tmap_a,
           }
           if (ncols > 0) {
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
-              float4 o;
-              o.x = __uint_as_float(v[4 * q]) * scale;
-              o.y = __uint_as_float(v[4 * q + 1]) * scale;
-              o.z = __uint_as_float(v[4 * q + 2]) * scale;
-              o.w = __uint_as_float(v[4 * q + 3]) * scale;
-              amax = fmaxf(amax, fmaxf(fmaxf(fabsf(o.x), fabsf(o.y)), fmaxf(fabsf(o.z), fabsf(o.w))));
-              reinterpret_cast<float4*>(dst + 64 * h2)[q] = o;
+            for (int q = 0; q < 8; ++q) {
+              float o[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                o[e] = __uint_as_float(v[8 * q + e]) * scale;
+                amax = fmaxf(amax, fabsf(o[e]));
+              }
+              float* d = dst + 64 * h2 + 8 * q;
+              if (wide_st) {
+                st_global_v8(d, __float_as_uint(o[0]), __float_as_uint(o[1]), __float_as_uint(o[2]),
+                             __float_as_uint(o[3]), __float_as_uint(o[4]), __float_as_uint(o[5]),
+                             __float_as_uint(o[6]), __float_as_uint(o[7]));
+              } else {
+                reinterpret_cast<float4*>(d)[0] = make_float4(o[0], o[1], o[2], o[3]);
+                reinterpret_cast<float4*>(d)[1] = make_float4(o[4], o[5], o[6], o[7]);
+              }
             }
           }
         }
