@@ -84,8 +84,6 @@ struct GemmArgs {
   uint32_t* status;
 };
 fp4_status gemm_launch(const GemmArgs& g, cudaStream_t s);
-// CTA-pair (cta_group::2) variant, 256 x 256 tiles (gemm_pair.cu).
-fp4_status gemm_launch_pair(const GemmArgs& g, cudaStream_t s);
 // Scale factors staged into TMEM by tcgen05.st warps (gemm_sfst.cu).
 fp4_status gemm_launch_sfst(const GemmArgs& g, cudaStream_t s);
 
