@@ -43,6 +43,19 @@ FP4_PER_BF16 = 4.0          # nominal dense FP4 / dense BF16 tensor throughput (
 Q_BYTES_PER_ELEM = 2 + 2 + 2 * (0.5 + 1 / 16)
 
 
+def max_over_ranks(x: float, device, world: int) -> float:
+    """The largest of every rank's `x` (all ranks take part; any backend)."""
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Units processed by all ranks per second, timed by the slowest rank."""
+    return world * units_per_rank / (ms_max * 1e-3)
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -306,10 +319,7 @@ def run_ours(args, rank, world, device):
     if world > 1:
         torch.distributed.barrier()
     ms = t0.elapsed_time(t1) / args.steps
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = max_over_ranks(ms, device, world)
     assert ws.status() == 0, f"device status {ws.status()}"
 
     ev = [(kind, units, a, b) for per in evs for (kind, units, _f, _l), (a, b) in zip(calls, per)]
@@ -342,17 +352,15 @@ def run_ours(args, rank, world, device):
     e2e = None
     if not args.no_e2e:
         e_ms, h2d, d2h = e2e_run(F, layers, cache, cfg, ws, args.e2e_steps, device)
-        e_ms_t = torch.tensor([e_ms], dtype=torch.float64, device=device)
-        if world > 1:
-            torch.distributed.all_reduce(e_ms_t, op=torch.distributed.ReduceOp.MAX)
-        e2e = {"value": round(world * flops_step / (float(e_ms_t.item()) * 1e-3) / 1e12, 2),
+        e_max = max_over_ranks(e_ms, device, world)
+        e2e = {"value": round(whole_job_rate(flops_step, world, e_max) / 1e12, 2),
                "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": round(float(e_ms_t.item()), 3),
+               "ms_per_step": round(e_max, 3),
                "api": "fqt_linear_fwd + fqt_linear_bwd, host buffers"}
 
     out = {
         "metric": METRIC,
-        "value": round(world * flops_step / (ms_max * 1e-3) / 1e12, 2),
+        "value": round(whole_job_rate(flops_step, world, ms_max) / 1e12, 2),
         "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms_max, 3),
@@ -412,6 +420,65 @@ def run_reference(args):
                     "d2h_bytes_per_step": 0}}
 
 
+# Quantizer sweep: (name, format, block, rounding, Hadamard points, algorithmic
+# bytes per element).  One output (row-wise), tensor-core scale layout only,
+# amax computed in the call: 2 B amax read + 2 B encode read + 0.5 B codes +
+# 1/16 B scales (NVFP4; the 16x16 tile scale is written once per row of its
+# tile in that layout); MXFP4 needs no amax pass: 2 + 0.5 + 1/32.
+SWEEP_MODES = [
+    ("nvfp4_1x16_rtn", "nvfp4", "1d", "rtn", 0, 4.5625),
+    ("nvfp4_1x16_sr", "nvfp4", "1d", "sr", 0, 4.5625),
+    ("nvfp4_1x16_rtn_rht16", "nvfp4", "1d", "rtn", 16, 4.5625),
+    ("nvfp4_1x16_sr_rht16", "nvfp4", "1d", "sr", 16, 4.5625),
+    ("nvfp4_16x16_rtn", "nvfp4", "2d", "rtn", 0, 4.5625),
+    ("mxfp4_1x32_rtn", "mxfp4", "1d", "rtn", 0, 2.53125),
+    ("mxfp4_1x32_rtn_rht32", "mxfp4", "1d", "rtn", 32, 2.53125),
+]
+
+
+def run_sweep(args, device):
+    """Quantizer sweep over 2^n elements shaped [2^n / 4096, 4096], N(0,1) with
+    0.1 % of the elements x100; each timed call follows a 256 MiB write that
+    evicts L2; median of the repetitions."""
+    import fp4_fully_quantized_b200 as F
+    import fqt_synth as S
+    F.load()
+    ws = F.Workspace(device=device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    lines = []
+    for n in range(args.sweep_min, args.sweep_max + 1):
+        rows, cols = (1 << n) // 4096, 4096
+        x = S.sweep_tensor(n, seed=n, width=cols).to(device)
+        for name, fmt_s, blk_s, rnd_s, rht, bpe in SWEEP_MODES:
+            fmt = F.MXFP4 if fmt_s == "mxfp4" else F.NVFP4
+            blk = F.BLOCK_2D if blk_s == "2d" else F.BLOCK_1D
+            q = F.QTensor.empty(rows, cols, fmt, blk, device=device, logical_scales=False)
+            fn = lambda: F.fp4_quantize(x, q, fmt=fmt, block=blk,
+                                        round=F.SR if rnd_s == "sr" else F.RTN, rht_n=rht,
+                                        rht_seed=7, sr_seed=11, sr_stream=1, ws=ws)
+            reps = 20 if n < 28 else 5
+            for _ in range(3):
+                fn()
+            times = []
+            for _ in range(reps):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                fn()
+                b.record()
+                torch.cuda.synchronize()
+                times.append(a.elapsed_time(b))
+            assert ws.status() == 0, f"device status {ws.status()}"
+            ms = statistics.median(times)
+            gbs = rows * cols * bpe / (ms * 1e-3) / 1e9
+            lines.append({"case": "sweep", "mode": name, "log2_elems": n, "rows": rows,
+                          "cols": cols, "ms": round(ms, 5), "bytes_per_elem": bpe,
+                          "rate": round(gbs, 1), "unit": "GB/s"})
+            del q
+        del x
+    return lines
+
+
 def run_case(args, device):
     """A single kernel family on one small problem (for profiler captures):
     --case gemm: NVFP4 fprop-style GEMM [m, k] x [n, k]^T, BF16 out;
@@ -456,8 +523,11 @@ def run_case(args, device):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--case", choices=["gemm", "quant", "quant_sr"], default=None,
-                    help="time one kernel family on a small problem (profiling)")
+    ap.add_argument("--case", choices=["gemm", "quant", "quant_sr", "sweep"], default=None,
+                    help="time one kernel family on one problem (profiling), or the "
+                         "quantizer sweep over 2^n elements")
+    ap.add_argument("--sweep-min", type=int, default=20)
+    ap.add_argument("--sweep-max", type=int, default=30)
     ap.add_argument("--m", type=int, default=8192)
     ap.add_argument("--n", type=int, default=4096)
     ap.add_argument("--k", type=int, default=4096)
@@ -482,7 +552,11 @@ def main():
     if args.case is not None:
         dev = torch.device("cuda", local)
         torch.cuda.set_device(dev)
-        print(json.dumps(run_case(args, dev)), flush=True)
+        if args.case == "sweep":
+            for line in run_sweep(args, dev):
+                print(json.dumps(line), flush=True)
+        else:
+            print(json.dumps(run_case(args, dev)), flush=True)
         return
 
     if args.impl == "reference":
