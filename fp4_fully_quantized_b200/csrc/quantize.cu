@@ -147,23 +147,36 @@ amax_plain_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t col
 }
 
 // ---------------------------------------------------------------------------
-// Row-wise quantization (NVFP4 BS = 16 or MXFP4 BS = 32).
+// Row-wise quantization (NVFP4 BS = 16 or MXFP4 BS = 32).  A warp takes one
+// row segment of 32 x kRowChunks 16-byte chunks (1024 elements): lane l owns
+// chunks l, l + 32, ... of the segment, all of whose loads are issued before
+// any is encoded; the lanes of a block (2 for NVFP4, 4 for MXFP4) are
+// adjacent, so the block max and the Hadamard stages are warp shuffles.
+// NVFP4 reads RN(s_enc / value(sf)) from a per-CTA table of the 128 E4M3
+// codes instead of dividing per block.
 // ---------------------------------------------------------------------------
+constexpr int kRowChunks = 4;
+
 template <int BS, int RHT_N, bool SR>
 __global__ void __launch_bounds__(kThreads)
 quant_rows_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
-                  uint32_t rht_mask, uint64_t sr_seed, uint32_t sr_stream,
+                  uint32_t rht_mask, const __grid_constant__ PhiloxKeys K, uint32_t sr_stream,
                   const float* __restrict__ amax_src, float* amax_out, float* s_dec_out,
                   uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
                   uint8_t* __restrict__ scales_mma, uint32_t* status) {
   constexpr bool NV = (BS == 16);
-  constexpr int TPB = BS / 8;                 // threads per block
-  const int64_t cpr = cols >> 3, total = rows * cpr;
-  const int64_t S = cols / BS;
+  constexpr int TPB = BS / 8;                 // lanes per block
+  constexpr int SEG = 32 * kRowChunks;        // chunks per warp step
+  const int64_t cpr = cols >> 3;              // 16-byte chunks per row
+  const int64_t segs = (cpr + SEG - 1) / SEG; // warp steps per row
+  const int64_t units = rows * segs;
+  const int64_t S = cols / BS, S4 = (S + 3) & ~3LL;
   const int lane = threadIdx.x & 31;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
 
   float s_enc = 1.0f, s_dec = 1.0f;
+  __shared__ float inv_tab[128];
   if constexpr (NV) {
     const float A = *amax_src;
     if (!(A <= FLT_MAX)) {                    // Inf or NaN: precondition violated
@@ -173,62 +186,67 @@ quant_rows_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t col
     if (blockIdx.x == 0 && threadIdx.x == 0) {
       if (amax_out != nullptr && amax_out != amax_src) *amax_out = A;
     }
+    for (int c = threadIdx.x; c < 128; c += blockDim.x)
+      inv_tab[c] = (c == 0 || c == 127) ? 0.0f : fminf(__fdiv_rn(s_enc, e4m3_value((uint32_t)c)), FLT_MAX);
+    __syncthreads();
   }
   if (blockIdx.x == 0 && threadIdx.x == 0 && s_dec_out != nullptr) *s_dec_out = s_dec;
 
-  for (int64_t g0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x - lane); g0 < total;
-       g0 += stride) {
-    const int64_t g = g0 + lane;
-    const bool active = g < total;
-    const int64_t r = active ? g / cpr : 0, j = active ? g - r * cpr : 0;
-    float v[8];
-    if (active) {
-      bf16x8_to_f32(ld_nc_v4(x + r * ld + j * 8), v);
-    } else {
+  for (int64_t u = warp0; u < units; u += nwarps) {
+    const int64_t r = u / segs;
+    const int64_t c0 = (u - r * segs) * SEG;
+    const __nv_bfloat16* xr = x + r * ld;
+    uint4 raw[kRowChunks];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-    }
-    if constexpr (RHT_N > 0) rht_chunk<RHT_N>(v, rht_mask, (int)(j % (RHT_N / 8)));
-
-    float bmax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
-#pragma unroll
-    for (int lx = 1; lx < TPB; lx <<= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xFFFFFFFFu, bmax, lx));
-
-    uint32_t sf;
-    float inv;
-    if constexpr (NV) {
-      const float t = __fdiv_rn(__fmul_rn(bmax, s_enc), 6.0f);
-      sf = e4m3_rn_sat(t);
-      inv = (sf == 0) ? 0.0f : fminf(__fdiv_rn(s_enc, e4m3_value(sf)), FLT_MAX);
-    } else {
-      int e = (bmax == 0.0f) ? -127 : floor_log2_f32(bmax) - 2;
-      e = max(-127, min(127, e));
-      sf = (uint32_t)(e + 127);
-      inv = exp2_neg_exact(e);
+    for (int q = 0; q < kRowChunks; ++q) {
+      const int64_t c = c0 + 32 * q + lane;
+      raw[q] = (c < cpr) ? ld_nc_v4(xr + c * 8) : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], inv);
-
-    uint32_t packed;
-    if constexpr (!SR) {
-      packed = e2m1x8_rn(v);
-    } else {
-      const uint64_t i0 = (uint64_t)r * (uint64_t)cols + (uint64_t)(j * 8);
-      const U4 w0 = philox4x32_10(i0 >> 2, sr_stream, sr_seed);
-      const U4 w1 = philox4x32_10((i0 >> 2) + 1, sr_stream, sr_seed);
-      const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-      packed = 0;
+    for (int q = 0; q < kRowChunks; ++q) {
+      const int64_t c = c0 + 32 * q + lane;
+      if (c0 + 32 * q >= cpr) break;          // warp-uniform: the segment's tail is done
+      float v[8];
+      bf16x8_to_f32(raw[q], v);
+      if constexpr (RHT_N > 0) rht_chunk<RHT_N>(v, rht_mask, lane % (RHT_N / 8));
+      float bmax = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) packed |= e2m1_sr(v[i], u[i]) << (4 * i);
-    }
-    if (active) {
-      *reinterpret_cast<uint32_t*>(codes + r * (cols >> 1) + j * 4) = packed;
-      if ((j % TPB) == 0) {
-        const int64_t s = j / TPB;
-        if (scales != nullptr) scales[r * S + s] = (uint8_t)sf;
-        if (scales_mma != nullptr) scales_mma[mma_sf_offset(r, s, (S + 3) & ~3LL)] = (uint8_t)sf;
+      for (int i = 0; i < 8; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
+#pragma unroll
+      for (int lx = 1; lx < TPB; lx <<= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xFFFFFFFFu, bmax, lx));
+      uint32_t sf;
+      float inv;
+      if constexpr (NV) {
+        const float t = __fdiv_rn(__fmul_rn(bmax, s_enc), 6.0f);
+        sf = e4m3_rn_sat(t);                  // 0 .. 126
+        inv = inv_tab[sf];
+      } else {
+        int e = (bmax == 0.0f) ? -127 : floor_log2_f32(bmax) - 2;
+        e = max(-127, min(127, e));
+        sf = (uint32_t)(e + 127);
+        inv = exp2_neg_exact(e);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], inv);
+      uint32_t packed;
+      if constexpr (!SR) {
+        packed = e2m1x8_rn(v);
+      } else {
+        const uint64_t i0 = (uint64_t)r * (uint64_t)cols + (uint64_t)(c * 8);
+        const U4 w0 = philox_keyed(i0 >> 2, sr_stream, K);
+        const U4 w1 = philox_keyed((i0 >> 2) + 1, sr_stream, K);
+        const uint32_t ud[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        packed = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) packed += e2m1_sr(v[i], ud[i]) << (4 * i);
+      }
+      if (c < cpr) {
+        *reinterpret_cast<uint32_t*>(codes + r * (cols >> 1) + c * 4) = packed;
+        if ((lane % TPB) == 0) {
+          const int64_t sb = c / TPB;
+          if (scales != nullptr) scales[r * S + sb] = (uint8_t)sf;
+          if (scales_mma != nullptr) scales_mma[mma_sf_offset(r, sb, S4)] = (uint8_t)sf;
+        }
       }
     }
   }
@@ -778,7 +796,7 @@ cudaError_t launch_amax_cols(const void* x, int64_t rows, int64_t cols, int64_t 
 template <int BS, int RHT_N, bool SR>
 static void rows_variant(const RowQuantArgs& a, int grid, cudaStream_t s) {
   quant_rows_kernel<BS, RHT_N, SR><<<grid, kThreads, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(a.x), a.rows, a.cols, a.ld, a.rht_mask, a.sr_seed,
+      static_cast<const __nv_bfloat16*>(a.x), a.rows, a.cols, a.ld, a.rht_mask, philox_keys(a.sr_seed),
       a.sr_stream, a.amax_src, a.amax_out, a.s_dec, a.codes, a.scales, a.scales_mma, a.status);
 }
 
@@ -804,7 +822,8 @@ static void cols_variant(const RowQuantArgs& a, int grid, cudaStream_t s) {
   } while (0)
 
 cudaError_t launch_quant_rows(const RowQuantArgs& a, cudaStream_t s) {
-  const int grid = grid_for(a.rows * (a.cols / 8), kThreads, 8);
+  const int64_t segs = ((a.cols / 8) + 32 * kRowChunks - 1) / (32 * kRowChunks);
+  const int grid = grid_for(a.rows * segs, kThreads / 32, 8);
   FP4_DISPATCH(rows_variant, a, grid, s);
   count_launches(1);
   return cudaGetLastError();
