@@ -479,6 +479,144 @@ def run_sweep(args, device):
     return lines
 
 
+def run_swiglu(device, layers=8, hidden=2048, ffn=8192, tokens=16384, seed=0, check_rows=8):
+    """Chained SwiGLU MLP stack through the library's linear layer: NVFP4 fprop
+    through all layers (RTN, 16x16 weight tiles), then dgrad / wgrad back with
+    stochastically rounded gradients.  Every linear is fqt_linear_fwd /
+    fqt_linear_bwd; the SwiGLU glue, silu(g) * u and its derivative, is harness
+    code (torch, FP32 math on BF16 tensors).  The same stack in unquantized FP32
+    is the comparison.  Returns per-layer relative Frobenius errors of the
+    activations, input gradients and both weight gradients, the device time of
+    the quantized pass, and the oracle spot check of the first and last layers'
+    quantized operands (sampled rows, codes and scales bit-exact)."""
+    import fp4_fully_quantized_b200 as F
+    import fqt_synth as S
+    F.load()
+    L, H, Fd, M = layers, hidden, ffn, tokens
+    cfg = F.linear_cfg(F.NVFP4, out_dtype=F.OUT_BF16, seed=seed)
+    w_gu = [S.normal((2 * Fd, H), 0.02, seed=100 + l).to(device) for l in range(L)]
+    w_d = [S.normal((H, Fd), 0.02, seed=200 + l).to(device) for l in range(L)]
+    x0 = S.normal((M, H), 1.0, seed=1).to(device)
+    dy_top = S.normal((M, H), 1e-3, seed=2).to(device)
+    ws = F.Workspace(M, 2 * Fd, max(H, Fd), device=device)
+    chk = {0, L - 1}
+    sv_gu = [F.Saved.empty(M, 2 * Fd, H, cfg, device, logical_scales=l in chk) for l in range(L)]
+    sv_d = [F.Saved.empty(M, H, Fd, cfg, device, logical_scales=l in chk) for l in range(L)]
+
+    def silu(g):
+        return g * torch.sigmoid(g)
+
+    def dsilu(g):
+        sg = torch.sigmoid(g)
+        return sg * (1 + g * (1 - sg))
+
+    # ---- quantized stack
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record()
+    h, acts, gus, hin = x0, [], [], []
+    for l in range(L):
+        hin.append(h)
+        y = torch.empty((M, 2 * Fd), dtype=torch.bfloat16, device=device)
+        F.fqt_linear_fwd(cfg, h, w_gu[l], y, sv_gu[l], ws)
+        gu = y.float()
+        gus.append(gu)
+        a = (silu(gu[:, :Fd]) * gu[:, Fd:]).to(torch.bfloat16).contiguous()
+        hin.append(a)
+        h = torch.empty((M, H), dtype=torch.bfloat16, device=device)
+        F.fqt_linear_fwd(cfg, a, w_d[l], h, sv_d[l], ws)
+        acts.append(h)
+    d, dxs, dwg, dwd, dys = dy_top, [None] * L, [None] * L, [None] * L, {}
+    for l in reversed(range(L)):
+        dys[(l, "d")] = d
+        da = torch.empty((M, Fd), dtype=torch.bfloat16, device=device)
+        dwd[l] = torch.empty((H, Fd), dtype=torch.float32, device=device)
+        F.fqt_linear_bwd(cfg, d, sv_d[l], da, dwd[l], ws)
+        g, u = gus[l][:, :Fd], gus[l][:, Fd:]
+        daf = da.float()
+        dgu = torch.cat([daf * u * dsilu(g), daf * silu(g)], dim=1).to(torch.bfloat16).contiguous()
+        dys[(l, "gu")] = dgu
+        dx = torch.empty((M, H), dtype=torch.bfloat16, device=device)
+        dwg[l] = torch.empty((2 * Fd, H), dtype=torch.float32, device=device)
+        F.fqt_linear_bwd(cfg, dgu, sv_gu[l], dx, dwg[l], ws)
+        dxs[l] = dx
+        d = dx
+    t1.record()
+    torch.cuda.synchronize()
+    assert ws.status() == 0, f"device status {ws.status()}"
+    ms = t0.elapsed_time(t1)
+
+    # ---- FP32 reference stack (no quantization, no BF16 rounding in between)
+    prev_tf32 = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = False
+    try:
+        hr, racts, rgus, rins = x0.float(), [], [], []
+        for l in range(L):
+            rins.append(hr)
+            gu = hr @ w_gu[l].float().t()
+            rgus.append(gu)
+            a = silu(gu[:, :Fd]) * gu[:, Fd:]
+            rins.append(a)
+            hr = a @ w_d[l].float().t()
+            racts.append(hr)
+        dr = dy_top.float()
+        rdx, rdwg, rdwd = [None] * L, [None] * L, [None] * L
+        for l in reversed(range(L)):
+            rdwd[l] = dr.t() @ rins[2 * l + 1]
+            da = dr @ w_d[l].float()
+            g, u = rgus[l][:, :Fd], rgus[l][:, Fd:]
+            dgu = torch.cat([da * u * dsilu(g), da * silu(g)], dim=1)
+            rdwg[l] = dgu.t() @ rins[2 * l]
+            dr = dgu @ w_gu[l].float()
+            rdx[l] = dr
+        # the same forward stack with every GEMM input and output rounded to
+        # BF16 (no FP4): the stack's own amplification of small rounding errors
+        hb, bacts = x0.float(), []
+        for l in range(L):
+            gu = (hb @ w_gu[l].float().t()).to(torch.bfloat16).float()
+            a = (silu(gu[:, :Fd]) * gu[:, Fd:]).to(torch.bfloat16).float()
+            hb = (a @ w_d[l].float().t()).to(torch.bfloat16).float()
+            bacts.append(hb)
+    finally:
+        torch.backends.cuda.matmul.allow_tf32 = prev_tf32
+
+    def rel(a, b):
+        return float((a.float() - b).norm() / b.norm())
+
+    per_layer = [{"layer": l + 1, "act": round(rel(acts[l], racts[l]), 5),
+                  "act_bf16_only": round(rel(bacts[l], racts[l]), 5),
+                  "dx": round(rel(dxs[l], rdx[l]), 5),
+                  "dw_gate_up": round(rel(dwg[l], rdwg[l]), 5),
+                  "dw_down": round(rel(dwd[l], rdwd[l]), 5)} for l in range(L)]
+
+    # ---- oracle spot check: sampled rows of the first and last layers'
+    # quantized X (RTN) and dY (SR), codes and logical scales bit-exact
+    import oracle as O
+    rng = np.random.default_rng(seed + 7)
+    mism = 0
+    checked = 0
+    for l in sorted(chk):
+        for sv, xin, dyin in ((sv_gu[l], hin[2 * l], dys[(l, "gu")]), (sv_d[l], hin[2 * l + 1], dys[(l, "d")])):
+            for q, src, rnd, stream in ((sv.xq, xin, "rtn", 0), (sv.dyq, dyin, "sr", 1)):
+                rows_ = np.sort(rng.choice(M, check_rows, replace=False))
+                amax = float(q.amax.item())
+                C_ = src.shape[1]
+                codes = q.codes.view(M, C_ // 2)
+                scales = q.scales.view(M, C_ // 16)
+                for r in rows_:
+                    xr = src[int(r):int(r) + 1].float().cpu().numpy()
+                    ref = O.nvfp4_quantize_1d(xr, round_mode=rnd, sr_seed=seed, sr_stream=stream,
+                                              amax_in=amax, row_offset=int(r))
+                    mism += int((codes[int(r)].cpu().numpy() != ref["codes"][0]).sum())
+                    mism += int((scales[int(r)].cpu().numpy() != ref["scales"][0]).sum())
+                    checked += 1
+    return {"case": "swiglu", "layers": L, "hidden": H, "ffn": Fd, "tokens": M,
+            "ms_quantized_fwd_bwd": round(ms, 3),
+            "tflops_gemm_equiv": round(L * 6 * M * (2 * Fd * H + H * Fd) / (ms * 1e-3) / 1e12, 1),
+            "rel_err_vs_fp32": per_layer, "oracle_rows_checked": checked,
+            "oracle_mismatches": mism}
+
+
 def run_case(args, device):
     """A single kernel family on one small problem (for profiler captures):
     --case gemm: NVFP4 fprop-style GEMM [m, k] x [n, k]^T, BF16 out;
@@ -523,7 +661,7 @@ def run_case(args, device):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--case", choices=["gemm", "quant", "quant_sr", "sweep"], default=None,
+    ap.add_argument("--case", choices=["gemm", "quant", "quant_sr", "sweep", "swiglu"], default=None,
                     help="time one kernel family on one problem (profiling), or the "
                          "quantizer sweep over 2^n elements")
     ap.add_argument("--sweep-min", type=int, default=20)
@@ -555,6 +693,8 @@ def main():
         if args.case == "sweep":
             for line in run_sweep(args, dev):
                 print(json.dumps(line), flush=True)
+        elif args.case == "swiglu":
+            print(json.dumps(run_swiglu(dev, seed=args.seed)), flush=True)
         else:
             print(json.dumps(run_case(args, dev)), flush=True)
         return

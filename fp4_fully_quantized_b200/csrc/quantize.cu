@@ -427,22 +427,32 @@ quant_2d_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols,
     if (amax_out_t && amax_out_t != amax_src) *amax_out_t = A;
   }
 
-  for (int64_t tid = blockIdx.x; tid < tiles_r * tiles_c; tid += gridDim.x) {
+  // The next tile's two 16-byte loads per thread are issued before the
+  // current tile is encoded, so their latency overlaps the encode.
+  const int64_t ntiles = tiles_r * tiles_c;
+  auto load_tile = [&](int64_t tid, uint4* raw) {
     const int64_t r0 = (tid / tiles_c) * kTile, c0 = (tid % tiles_c) * kTile;
-    __syncthreads();
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+      const int rr = (t >> 3) + 32 * it, cc = (t & 7) * 8;
+      raw[it] = (r0 + rr < rows && c0 + cc < cols) ? ld_nc_v4(x + (r0 + rr) * ld + c0 + cc)
+                                                  : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  uint4 nxt[2];
+  if (blockIdx.x < ntiles) load_tile(blockIdx.x, nxt);
+  for (int64_t tid = blockIdx.x; tid < ntiles; tid += gridDim.x) {
+    const int64_t r0 = (tid / tiles_c) * kTile, c0 = (tid % tiles_c) * kTile;
+    __syncthreads();                          // the previous tile's reads are done
 #pragma unroll
     for (int it = 0; it < 2; ++it) {
       const int rr = (t >> 3) + 32 * it, cc = (t & 7) * 8;
       float v[8];
-      if (r0 + rr < rows && c0 + cc < cols) {
-        bf16x8_to_f32(ld_nc_v4(x + (r0 + rr) * ld + c0 + cc), v);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-      }
+      bf16x8_to_f32(nxt[it], v);
 #pragma unroll
       for (int i = 0; i < 8; ++i) tile[rr][cc + i] = v[i];
     }
+    if (tid + gridDim.x < ntiles) load_tile(tid + gridDim.x, nxt);
     __syncthreads();
     {  // tile max: 16 threads per 16x16 tile, one tile row each
       const int q = t >> 4, rr = t & 15;
