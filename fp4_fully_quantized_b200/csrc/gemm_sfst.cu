@@ -258,21 +258,23 @@ fp4_gemm_sfst_kernel(const __grid_constant__ CUtensorMap tmap_a,
       const int ncols = min(BN / 2, p.N - nb * BN - c_begin);
       const int64_t col = (int64_t)nb * BN + c_begin;
       const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)c_begin;
-      uint32_t r[32];
       if (!p.out_f32) {
-        // drain 128 columns, packing to BF16 as they arrive (64 registers)
+        // drain 128 columns in two 64-column loads, packing to BF16 as they
+        // arrive (64 registers); two TMEM round trips before the release
         uint32_t pk[64];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          tmem_ld32_nowait(taddr + 32 * q, r);
+        for (int q = 0; q < 2; ++q) {
+          uint32_t r2[64];
+          tmem_ld32_nowait(taddr + 64 * q, r2);
+          tmem_ld32_nowait(taddr + 64 * q + 32, r2 + 32);
           asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-          for (int h = 0; h < 16; ++h) {
-            const float a0 = __uint_as_float(r[2 * h]) * scale;
-            const float a1 = __uint_as_float(r[2 * h + 1]) * scale;
+          for (int h = 0; h < 32; ++h) {
+            const float a0 = __uint_as_float(r2[2 * h]) * scale;
+            const float a1 = __uint_as_float(r2[2 * h + 1]) * scale;
             amax = fmaxf(amax, fmaxf(fabsf(a0), fabsf(a1)));
             __nv_bfloat162 b2 = __floats2bfloat162_rn(a0, a1);
-            memcpy(&pk[16 * q + h], &b2, 4);
+            memcpy(&pk[32 * q + h], &b2, 4);
           }
         }
         tc_fence_before();

@@ -82,25 +82,32 @@ template <int RHT_N>
 __global__ void __launch_bounds__(kThreads)
 amax_rows_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
                  uint32_t rht_mask, float* amax) {
-  const int64_t cpr = cols >> 3, total = rows * cpr;
+  // one warp per row segment of 32 x 4 16-byte chunks, all four loads in
+  // flight before the rotation (the lanes of a Hadamard block are adjacent)
+  constexpr int CH = 4, SEG = 32 * CH;
+  const int64_t cpr = cols >> 3;
+  const int64_t segs = (cpr + SEG - 1) / SEG, units = rows * segs;
   const int lane = threadIdx.x & 31;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   float m = 0.0f;
-  for (int64_t g0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x - lane); g0 < total;
-       g0 += stride) {
-    const int64_t g = g0 + lane;
-    float v[8];
-    if (g < total) {
-      const int64_t r = g / cpr, j = g - r * cpr;
-      bf16x8_to_f32(ld_nc_v4(x + r * ld + j * 8), v);
-      if constexpr (RHT_N > 0) rht_chunk<RHT_N>(v, rht_mask, (int)(j % (RHT_N / 8)));
-    } else {
+  for (int64_t u = warp0; u < units; u += nwarps) {
+    const int64_t r = u / segs, c0 = (u - r * segs) * SEG;
+    const __nv_bfloat16* xr = x + r * ld;
+    uint4 raw[CH];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-      if constexpr (RHT_N > 0) rht_chunk<RHT_N>(v, rht_mask, 0);
+    for (int q = 0; q < CH; ++q) {
+      const int64_t c = c0 + 32 * q + lane;
+      raw[q] = (c < cpr) ? ld_nc_v4(xr + c * 8) : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) m = absmax_keep_nan(m, v[i]);
+    for (int q = 0; q < CH; ++q) {
+      float v[8];
+      bf16x8_to_f32(raw[q], v);
+      if constexpr (RHT_N > 0) rht_chunk<RHT_N>(v, rht_mask, lane % (RHT_N / 8));
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m = absmax_keep_nan(m, v[i]);
+    }
   }
   block_amax_atomic(m, amax);
 }
@@ -780,7 +787,8 @@ cudaError_t launch_amax_rows(const void* x, int64_t rows, int64_t cols, int64_t 
     count_launches(1);
     return cudaGetLastError();
   }
-  const int grid = grid_for(rows * (cols / 8), kThreads, 8);
+  const int64_t segs = ((cols / 8) + 32 * kRowChunks - 1) / (32 * kRowChunks);
+  const int grid = grid_for(rows * segs, kThreads / 32, 8);
   if (rht_n == 16) amax_rows_kernel<16><<<grid, kThreads, 0, s>>>(xp, rows, cols, ld, mask, amax);
   else if (rht_n == 32) amax_rows_kernel<32><<<grid, kThreads, 0, s>>>(xp, rows, cols, ld, mask, amax);
   else amax_rows_kernel<0><<<grid, kThreads, 0, s>>>(xp, rows, cols, ld, mask, amax);
