@@ -545,6 +545,16 @@ def run_swiglu(device, layers=8, hidden=2048, ffn=8192, tokens=16384, seed=0, ch
     torch.cuda.synchronize()
     assert ws.status() == 0, f"device status {ws.status()}"
     ms = t0.elapsed_time(t1)
+    # gradient norm against the SR quantization noise of each layer's dY
+    # (the two quantities the "FP4 All the Way" page relates)
+    sums = torch.zeros(2, dtype=torch.float64, device=device)
+    snr = {}
+    for l in range(L):
+        for key, sv in (("down", sv_d[l]), ("gate_up", sv_gu[l])):
+            g = dys[(l, "d" if key == "down" else "gu")]
+            F.fp4_quant_noise(g, sv.dyq, sums, ws)
+            sx, sn = sums.tolist()
+            snr[(l, key)] = (sx / sn) ** 0.5 if sn > 0 else float("inf")
 
     # ---- FP32 reference stack (no quantization, no BF16 rounding in between)
     prev_tf32 = torch.backends.cuda.matmul.allow_tf32
@@ -587,7 +597,9 @@ def run_swiglu(device, layers=8, hidden=2048, ffn=8192, tokens=16384, seed=0, ch
                   "act_bf16_only": round(rel(bacts[l], racts[l]), 5),
                   "dx": round(rel(dxs[l], rdx[l]), 5),
                   "dw_gate_up": round(rel(dwg[l], rdwg[l]), 5),
-                  "dw_down": round(rel(dwd[l], rdwd[l]), 5)} for l in range(L)]
+                  "dw_down": round(rel(dwd[l], rdwd[l]), 5),
+                  "grad_snr_dy_down": round(snr[(l, "down")], 3),
+                  "grad_snr_dy_gate_up": round(snr[(l, "gate_up")], 3)} for l in range(L)]
 
     # ---- oracle spot check: sampled rows of the first and last layers'
     # quantized X (RTN) and dY (SR), codes and logical scales bit-exact

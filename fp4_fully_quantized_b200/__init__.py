@@ -33,7 +33,8 @@ STATUS = {0: "FP4_OK", 1: "FP4_ERR_NULL", 2: "FP4_ERR_SHAPE", 3: "FP4_ERR_ALIGN"
 EXPORTS = ("fp4_qtensor_sizes", "fp4_qparams_default", "fp4_workspace_bytes", "fp4_quantize",
            "fp4_gemm", "fqt_linear_cfg_default", "fqt_linear_fwd", "fqt_linear_bwd",
            "fp4_read_device_status", "fp4_clear_device_status", "fp4_status_str",
-           "fp4_abi_version", "fp4_kernel_launches", "fp4_gemm_noalloc", "fp4_mma_rate")
+           "fp4_abi_version", "fp4_kernel_launches", "fp4_gemm_noalloc", "fp4_mma_rate",
+           "fp4_quant_noise")
 
 
 class Fp4Error(RuntimeError):
@@ -111,6 +112,8 @@ def load() -> C.CDLL:
     L.fp4_kernel_launches.argtypes = []
     L.fp4_mma_rate.restype = i32
     L.fp4_mma_rate.argtypes = [i32, i32, C.POINTER(C.c_float), vp, sz, vp]
+    L.fp4_quant_noise.restype = i32
+    L.fp4_quant_noise.argtypes = [vp, i64, i64, i64, C.POINTER(QTensorC), vp, vp, sz, vp]
     L.fp4_gemm_noalloc.restype = i32
     L.fp4_gemm_noalloc.argtypes = [C.POINTER(QTensorC), C.POINTER(QTensorC), C.c_float, vp, i64,
                                    i32, vp, vp]
@@ -255,6 +258,17 @@ def mma_rate(variant: int = 0, iters: int = 20000, stream=None) -> float:
     _check(load().fp4_mma_rate(variant, iters, C.byref(out), ws.ptr, ws.nbytes, _stream(stream)),
            "fp4_mma_rate")
     return float(out.value)
+
+
+def fp4_quant_noise(x: torch.Tensor, q: QTensor, sums: torch.Tensor, ws: Workspace | None = None,
+                    stream=None):
+    """sums[0] = sum x^2, sums[1] = sum (deq(q) - x)^2 (float64 CUDA tensor of 2)."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.is_cuda and x.stride(1) == 1
+    assert sums.dtype == torch.float64 and sums.numel() >= 2 and sums.is_cuda
+    code = load().fp4_quant_noise(_ptr(x), x.shape[0], x.shape[1], x.stride(0), C.byref(q.c),
+                                  _ptr(sums), ws.ptr if ws is not None else None,
+                                  ws.nbytes if ws is not None else 0, _stream(stream))
+    _check(code, "fp4_quant_noise")
 
 
 def linear_cfg(fmt: int = NVFP4, **overrides) -> LinearCfgC:

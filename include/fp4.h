@@ -247,6 +247,24 @@ fp4_status fqt_linear_bwd(const fqt_linear_cfg* cfg, int64_t M, int64_t N, int64
 fp4_status fp4_gemm_noalloc(const fp4_qtensor* a, const fp4_qtensor* b, float alpha, void* c,
                             int64_t ldc, int32_t out_dtype, float* c_amax, void* stream);
 
+/* Gradient-norm vs quantization-noise diagnostic ("FP4 All the Way" page,
+ * Summary: quantized training stops being effective below a threshold set
+ * by the relation between the gradient norm and the quantization noise; the
+ * page gives no formula, so this reports the two quantities themselves).
+ * With x the BF16 tensor [rows, cols] (leading dimension ld, ld % 8 == 0)
+ * and q its row-wise quantization (q->rows == rows, q->cols == cols, 1-D or
+ * 2-D NVFP4 or MXFP4, scales_mma or scales set):
+ *   sums[0] = sum x^2,  sums[1] = sum (deq(q) - x)^2,
+ *   deq(q) = e2m1(code) * block scale * s_dec(q)   (exact in double),
+ * accumulated in double.  `sums` is caller-owned device memory, two doubles,
+ * overwritten (zeroed first on `stream`).  The order of the additions is not
+ * fixed, so results agree with an exact sum to about 1e-12 relative.
+ * ||x|| / ||deq(q) - x|| = sqrt(sums[0] / sums[1]) is the signal-to-noise
+ * ratio of the quantized tensor. */
+fp4_status fp4_quant_noise(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                           const fp4_qtensor* q, double* sums, void* ws, size_t ws_bytes,
+                           void* stream);
+
 /* Synchronise `stream`, then return the device status word of `ws`
  * (FP4_OK when no device condition was recorded). */
 fp4_status fp4_read_device_status(const void* ws, void* stream);

@@ -7,9 +7,9 @@ its own CUDA implementation and shares no code with this one.
 The arithmetic lives in ``fp4_oracle.c`` (plain C, IEEE binary32, no FMA
 contraction); this module only marshals numpy arrays through ctypes.  The
 GEMM reference is a float64 matrix product (numpy ``@``) of the exactly
-dequantized operands, scaled afterwards by ``alpha * s_dec(a) * s_dec(b)``:
-"Matrix multiplications run on Tensor Cores in FP4, while accumulation
-happens in higher precision" ("FP4", Robots Atlas, How it works).
+dequantized operands, scaled afterwards by ``alpha * s_dec(a) * s_dec(b)``
+(the "FP4" page of Robots Atlas, How it works: the products are formed from
+FP4 operands and summed at a wider precision).
 
 Parity status of each function is recorded in the repository's design notes;
 the Philox generator is pinned statistically only (no published known-answer
@@ -258,6 +258,18 @@ def dequantize(codes, scales, block=(1, 16), e8m0: bool = False) -> np.ndarray:
     out = np.empty((R, half * 2), np.float64)
     lib().orc_dequantize(codes, scales, R, half * 2, block[0], block[1], int(e8m0), out)
     return out
+
+
+def quant_noise(x, codes, scales, s_dec: float, block=(1, 16), e8m0: bool = False):
+    """(sum x^2, sum (deq - x)^2) in float64 for a tensor x and its
+    quantization (codes, logical scales, per-tensor decode scale s_dec):
+    deq = e2m1(code) * block scale * s_dec.  The gradient-norm and
+    quantization-noise pair of the "FP4 All the Way" page (Summary), which
+    states a threshold between them without giving its form."""
+    x = np.asarray(x, dtype=np.float64)
+    deq = dequantize(codes, scales, block, e8m0) * float(s_dec)
+    d = deq - x
+    return float(np.sum(x * x)), float(np.sum(d * d))
 
 
 def gemm(a_hat: np.ndarray, b_hat: np.ndarray, alpha: float = 1.0, s_dec_a: float = 1.0,

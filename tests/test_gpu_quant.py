@@ -130,6 +130,37 @@ def test_mxfp4_rows_and_transposed(gpu_lib, shape, rnd, rht):
     _check_1d(qt, O.mxfp4_quantize(np.ascontiguousarray(xf.T), sr_stream=5, **kw), 1)
 
 
+@pytest.mark.parametrize("case", ["nvfp4_rtn", "nvfp4_sr", "nvfp4_2d", "mxfp4", "nvfp4_ragged"])
+def test_quant_noise_matches_oracle(gpu_lib, case):
+    """fp4_quant_noise (sum x^2, sum (deq - x)^2 in double) against the
+    oracle's float64 sums of the oracle's own quantization of the same x."""
+    F = gpu_lib
+    shape = (48, 80) if case == "nvfp4_ragged" else (256, 512)
+    x = S.sparse_outliers(*shape, seed=11)
+    xf = S.as_f32(x)
+    if case == "mxfp4":
+        q, _ = _gpu_quant(F, x, 1)
+        ref = O.mxfp4_quantize(xf)
+        want = O.quant_noise(xf, ref["codes"], ref["scales"], 1.0, block=(1, 32), e8m0=True)
+    elif case == "nvfp4_2d":
+        q, _ = _gpu_quant(F, x, 0, block=1)
+        ref = O.nvfp4_quantize_2d(xf)
+        want = O.quant_noise(xf, ref["codes"], ref["scales"], float(ref["s_dec"]), block=(16, 16))
+    else:
+        rnd = SR if case == "nvfp4_sr" else RTN
+        q, _ = _gpu_quant(F, x, 0, round=rnd, seed=5, stream=1)
+        ref = O.nvfp4_quantize_1d(xf, "sr" if rnd == SR else "rtn", sr_seed=5, sr_stream=1)
+        want = O.quant_noise(xf, ref["codes"], ref["scales"], float(ref["s_dec"]))
+    sums = torch.zeros(2, dtype=torch.float64, device="cuda")
+    ws = F.Workspace()
+    F.fp4_quant_noise(x.cuda(), q, sums, ws)
+    torch.cuda.synchronize()
+    got = sums.cpu().numpy()
+    assert got[0] == pytest.approx(want[0], rel=1e-12)
+    assert got[1] == pytest.approx(want[1], rel=1e-12)
+    assert 0.0 < got[1] < got[0]
+
+
 def test_edge_values(gpu_lib):
     F = gpu_lib
     rng = np.random.default_rng(0)

@@ -286,3 +286,48 @@ def test_nvfp4_reciprocal_saturates_for_subnormal_blocks():
     v = _e2m1(codes)
     assert np.isfinite(v).all() and (np.abs(v) <= 6).all()
     assert (np.sign(v[v != 0]) == np.sign(x[v != 0])).all()
+
+
+def test_quant_noise_closed_form_mxfp4_block():
+    """One MXFP4 block [4, 0.25, 1.25, 0, ...]: the block scale is 2^0 (max 4,
+    floor(log2 4) - 2 = 0); 0.25 and 1.25 are midpoints that round to the
+    even levels 0 and 1, each off by 0.25.  sum x^2 = 16 + 1/16 + 25/16,
+    sum noise^2 = 2/16."""
+    x = np.zeros((1, 32), np.float32)
+    x[0, :3] = [4.0, 0.25, 1.25]
+    q = O.mxfp4_quantize(x)
+    sx, sn = O.quant_noise(x, q["codes"], q["scales"], 1.0, block=(1, 32), e8m0=True)
+    assert sx == 17.625
+    assert sn == 0.125
+
+
+def test_quant_noise_zero_for_representable_blocks():
+    """Values already on the E2M1 grid of their block scale carry no noise."""
+    x = np.zeros((2, 32), np.float32)
+    x[0, :8] = [6, 4, 3, 2, 1.5, 1, 0.5, 0]
+    x[1, :8] = [-6, -3, -1, -0.5, 0.5, 1, 2, 4]
+    q = O.mxfp4_quantize(x)
+    sx, sn = O.quant_noise(x, q["codes"], q["scales"], 1.0, block=(1, 32), e8m0=True)
+    assert sn == 0.0
+    assert sx == float(np.sum(x.astype(np.float64) ** 2))
+
+
+def test_quant_noise_matches_independent_decode_nvfp4():
+    """NVFP4 with a tensor scale: the noise sum equals the one computed from
+    an independent decode (E2M1 levels from the page's level set, E4M3 block
+    scales through ml_dtypes) and is below the bound of half a level gap
+    (at most 1 in units of the block scale) per element."""
+    ml_dtypes = pytest.importorskip("ml_dtypes")
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal((8, 64)) * np.exp(rng.uniform(-3, 3, (8, 1)))).astype(np.float32)
+    q = O.nvfp4_quantize_1d(x)
+    sx, sn = O.quant_noise(x, q["codes"], q["scales"], float(q["s_dec"]))
+    codes = _codes(q["codes"])
+    vals = np.where(codes >= 8, -np.array(LEVELS)[codes & 7], np.array(LEVELS)[codes & 7])
+    sc = q["scales"].view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    deq = vals * np.repeat(sc, 16, axis=1) * float(q["s_dec"])
+    d = deq - x.astype(np.float64)
+    assert sx == pytest.approx(float(np.sum(x.astype(np.float64) ** 2)), rel=1e-15)
+    assert sn == pytest.approx(float(np.sum(d * d)), rel=1e-15)
+    gap_bound = np.repeat(sc, 16, axis=1) * float(q["s_dec"])      # half of the widest gap (2)
+    assert np.all(np.abs(d) <= gap_bound * (1 + 1e-6))
