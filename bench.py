@@ -37,6 +37,11 @@ LAYERS = [("qkvo", 4096, 4096)] * 4 + [("gate_up", 11008, 4096)] * 2 + [("down",
 METRIC = "NVFP4 linear fwd+bwd TFLOPS & % FP4 peak; quantizer GB/s & % HBM BW"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP4_PER_BF16 = 4.0          # nominal dense FP4 / dense BF16 tensor throughput (9 / 2.25 PF)
+# DRAM bytes (read + write) per GEMM launch, averaged over the 21 GEMM
+# launches of one step: ncu dram__bytes_read.sum + dram__bytes_write.sum
+# (single pass) of fp4_gemm_sfst_kernel as it stands, 344.9 MB read + 249.0 MB
+# written.  Set to None whenever the GEMM kernel changes until re-measured.
+GEMM_DRAM_BYTES_PER_LAUNCH = 5.939e8
 # Algorithmic bytes per element of one quantize call producing row-wise and
 # transposed outputs with an in-kernel amax: amax read 2 B + encode read 2 B
 # + two outputs of (0.5 B codes + 1/16 B scales).
@@ -379,7 +384,8 @@ def run_ours(args, rank, world, device):
                      "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1),
                      "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4),
                      "peak_source": f"{pk_src}: bf16 sustained x {FP4_PER_BF16:g} (nominal FP4/BF16)",
-                     "traffic": None, "launches": gemm_n,
+                     "traffic": GEMM_DRAM_BYTES_PER_LAUNCH, "traffic_unit": "bytes per launch (ncu)",
+                     "launches": gemm_n,
                      "avg_ms": round(gemm_ms / max(gemm_n, 1), 4),
                      "share_of_step": round(gemm_ms / (ms_max * args.steps), 3)},
         "quantizer": {"bound": "hbm", "achieved": round(q_gbs, 1), "peak": pk["hbm_gbs"],
@@ -643,10 +649,16 @@ def run_case(args, device):
     qa = F.QTensor.empty(M, K, device=device, logical_scales=False)
     qat = F.QTensor.empty(K, M, device=device, logical_scales=False)
     if args.case in ("quant", "quant_sr"):
-        r = F.SR if args.case == "quant_sr" else F.RTN
-        fn = lambda: F.fp4_quantize(x, qa, qat, round=r, round_t=F.SR, sr_seed=1, sr_stream=1,
-                                    sr_stream_t=3, ws=ws)
-        units, unit = M * K * Q_BYTES_PER_ELEM / 1e9, "GB/s"
+        rr, rc = (args.rounds or ("sr,sr" if args.case == "quant_sr" else "rtn,sr")).split(",")
+        r, rt = (F.SR if rr == "sr" else F.RTN), (F.SR if rc == "sr" else F.RTN)
+        amax_in = None
+        if args.amax_supplied:        # time the fused encode alone: amax computed once, then supplied
+            F.fp4_quantize(x, qa, qat, round=r, round_t=rt, sr_seed=1, sr_stream=1, sr_stream_t=3, ws=ws)
+            amax_in = qa.amax.clone()
+        fn = lambda: F.fp4_quantize(x, qa, qat, round=r, round_t=rt, sr_seed=1, sr_stream=1,
+                                    sr_stream_t=3, amax_in=amax_in, amax_in_t=amax_in, ws=ws)
+        bpe = Q_BYTES_PER_ELEM - (2 if args.amax_supplied else 0)
+        units, unit = M * K * bpe / 1e9, "GB/s"
     else:
         w = S.normal((N, K), 0.02, seed=2).to(device)
         qb = F.QTensor.empty(N, K, F.NVFP4, F.BLOCK_2D, device=device, logical_scales=False)
@@ -676,6 +688,10 @@ def main():
     ap.add_argument("--case", choices=["gemm", "quant", "quant_sr", "sweep", "swiglu"], default=None,
                     help="time one kernel family on one problem (profiling), or the "
                          "quantizer sweep over 2^n elements")
+    ap.add_argument("--rounds", default=None,
+                    help="--case quant: rounding of the row and transposed outputs, e.g. rtn,sr")
+    ap.add_argument("--amax-supplied", action="store_true",
+                    help="--case quant: supply the tensor amax (times the fused encode alone)")
     ap.add_argument("--sweep-min", type=int, default=20)
     ap.add_argument("--sweep-max", type=int, default=30)
     ap.add_argument("--m", type=int, default=8192)
