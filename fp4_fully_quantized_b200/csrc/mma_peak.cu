@@ -10,6 +10,9 @@
 //      K step needs
 //   2  cta_group::2, 256 x 256 x 64 per MMA (CTA pair)
 //   3  as 2, plus the scale-factor copies
+//   4  as 0, with the copies issued concurrently by a second warp (into a
+//      separate TMEM region) instead of by the MMA thread
+//   5  as 2, the same for the CTA pair
 // Operands are filled with pseudo-random codes and unit scales.  Waits are
 // bounded like the GEMM's.
 #include <cuda.h>
@@ -27,20 +30,20 @@ using namespace ptx;
 constexpr int A_BYTES = 128 * 128;      // 128 rows x 256 FP4
 constexpr int B_BYTES = 256 * 128;      // 256 rows (1 SM) / 128 rows per CTA (pair)
 constexpr int SF_BYTES = 3 * 512;
-constexpr int PEAK_SMEM = A_BYTES + B_BYTES + SF_BYTES + 1024 + 64;
+constexpr int PEAK_SMEM = A_BYTES + B_BYTES + SF_BYTES + 1024 + 64 + 16;
 
 __device__ __forceinline__ uint32_t hash32(uint32_t x) {
   x ^= x >> 16; x *= 0x7FEB352Du; x ^= x >> 15; x *= 0x846CA68Bu; x ^= x >> 16;
   return x;
 }
 
-template <bool PAIR, bool WITH_CP>
+template <bool PAIR, bool WITH_CP, bool CP_WARP = false>
 __device__ void peak_body(int iters, uint32_t* status, uint8_t* base) {
   uint8_t* sA = base;
   uint8_t* sB = base + A_BYTES;
   uint8_t* sSF = base + A_BYTES + B_BYTES;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sSF + SF_BYTES);
-  uint32_t* holder = reinterpret_cast<uint32_t*>(bar + 1);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sSF + SF_BYTES);   // [0] MMAs, [1] copier
+  uint32_t* holder = reinterpret_cast<uint32_t*>(bar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
   const int t = threadIdx.x;
   // random E2M1 codes (no NaN in FP4), unit E4M3 scales (0x38 = 1.0)
@@ -49,6 +52,7 @@ __device__ void peak_body(int iters, uint32_t* status, uint8_t* base) {
   for (int i = t; i < SF_BYTES; i += blockDim.x) sSF[i] = 0x38;
   if (t == 0) {
     mbar_init(smem_u32(bar), 1);
+    mbar_init(smem_u32(bar + 1), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -63,6 +67,27 @@ __device__ void peak_body(int iters, uint32_t* status, uint8_t* base) {
   tc_fence_after();
   const uint32_t tmem = *holder;
   const bool issuer = PAIR ? (cluster_ctarank() == 0 && t == 0) : (t == 0);
+  const bool copier = CP_WARP && (PAIR ? (cluster_ctarank() == 0 && t == 32) : (t == 32));
+  if (copier) {
+    // the copies of variant 1 / 3, from another warp, into columns 448+
+    const uint64_t sf0 = smem_desc(smem_u32(sSF), 0, 128, 0);
+    const uint64_t sf1 = smem_desc(smem_u32(sSF + 512), 0, 128, 0);
+    const uint64_t sf2 = smem_desc(smem_u32(sSF + 1024), 0, 128, 0);
+    const uint32_t t_cp = tmem + 448;
+    for (int i = 0; i < iters; ++i) {
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        if (PAIR) {
+          tc_cp_pair_32x128b(t_cp, sf0); tc_cp_pair_32x128b(t_cp + 4, sf1); tc_cp_pair_32x128b(t_cp + 8, sf2);
+        } else {
+          tc_cp_32x128b(t_cp, sf0); tc_cp_32x128b(t_cp + 4, sf1); tc_cp_32x128b(t_cp + 8, sf2);
+        }
+      }
+    }
+    if (PAIR) tc_commit_pair(smem_u32(bar + 1), 0x1);
+    else tc_commit(smem_u32(bar + 1));
+    mbar_wait(smem_u32(bar + 1), 0, abort_flag, status, 0x2001);
+  }
   if (issuer) {
     const uint32_t t_sfa = tmem + 256, t_sfb = tmem + 260;
     const uint64_t sf0 = smem_desc(smem_u32(sSF), 0, 128, 0);
@@ -102,19 +127,19 @@ __device__ void peak_body(int iters, uint32_t* status, uint8_t* base) {
   }
 }
 
-template <bool WITH_CP>
+template <bool WITH_CP, bool CP_WARP>
 __global__ void __launch_bounds__(128, 1) mma_peak_single(int iters, uint32_t* status) {
   extern __shared__ uint8_t sm[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm) + 1023) & ~uintptr_t(1023));
-  peak_body<false, WITH_CP>(iters, status, base);
+  peak_body<false, WITH_CP, CP_WARP>(iters, status, base);
 }
 
-template <bool WITH_CP>
+template <bool WITH_CP, bool CP_WARP>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1)
 mma_peak_pair(int iters, uint32_t* status) {
   extern __shared__ uint8_t sm[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm) + 1023) & ~uintptr_t(1023));
-  peak_body<true, WITH_CP>(iters, status, base);
+  peak_body<true, WITH_CP, CP_WARP>(iters, status, base);
 }
 
 }  // namespace
@@ -126,7 +151,7 @@ extern "C" fp4_status fp4_mma_rate(int32_t variant, int32_t iters, float* tflops
                                    void* ws, size_t ws_bytes, void* stream) {
   if (tflops_out == nullptr || ws == nullptr) return FP4_ERR_NULL;
   if (ws_bytes < sizeof(DeviceStatus)) return FP4_ERR_WORKSPACE;
-  if (variant < 0 || variant > 3 || iters <= 0) return FP4_ERR_SHAPE;
+  if (variant < 0 || variant > 5 || iters <= 0) return FP4_ERR_SHAPE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int grid = (sm_count() / 2) * 2;
   uint32_t* status = static_cast<uint32_t*>(ws);
@@ -134,14 +159,16 @@ extern "C" fp4_status fp4_mma_rate(int32_t variant, int32_t iters, float* tflops
   if (cudaEventCreate(&e0) != cudaSuccess || cudaEventCreate(&e1) != cudaSuccess) return FP4_ERR_CUDA;
   auto launch = [&]() {
     switch (variant) {
-      case 0: cudaFuncSetAttribute(mma_peak_single<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, PEAK_SMEM);
-              mma_peak_single<false><<<grid, 128, PEAK_SMEM, s>>>(iters, status); break;
-      case 1: cudaFuncSetAttribute(mma_peak_single<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, PEAK_SMEM);
-              mma_peak_single<true><<<grid, 128, PEAK_SMEM, s>>>(iters, status); break;
-      case 2: cudaFuncSetAttribute(mma_peak_pair<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, PEAK_SMEM);
-              mma_peak_pair<false><<<grid, 128, PEAK_SMEM, s>>>(iters, status); break;
-      default: cudaFuncSetAttribute(mma_peak_pair<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, PEAK_SMEM);
-               mma_peak_pair<true><<<grid, 128, PEAK_SMEM, s>>>(iters, status); break;
+#define FP4_PEAK_LAUNCH(KERN)                                                              \
+  cudaFuncSetAttribute(KERN, cudaFuncAttributeMaxDynamicSharedMemorySize, PEAK_SMEM);     \
+  KERN<<<grid, 128, PEAK_SMEM, s>>>(iters, status);
+      case 0: FP4_PEAK_LAUNCH((mma_peak_single<false, false>)); break;
+      case 1: FP4_PEAK_LAUNCH((mma_peak_single<true, false>)); break;
+      case 2: FP4_PEAK_LAUNCH((mma_peak_pair<false, false>)); break;
+      case 3: FP4_PEAK_LAUNCH((mma_peak_pair<true, false>)); break;
+      case 4: FP4_PEAK_LAUNCH((mma_peak_single<false, true>)); break;
+      default: FP4_PEAK_LAUNCH((mma_peak_pair<false, true>)); break;
+#undef FP4_PEAK_LAUNCH
     }
     count_launches(1);
   };
@@ -157,8 +184,9 @@ extern "C" fp4_status fp4_mma_rate(int32_t variant, int32_t iters, float* tflops
   cudaEventDestroy(e1);
   // flops: each CTA (single) or CTA pair issues iters * 4 MMAs of
   // 128x256x64 (single) or 256x256x64 (pair)
-  const double per_mma = (variant < 2) ? 2.0 * 128 * 256 * 64 : 2.0 * 256 * 256 * 64;
-  const double issuers = (variant < 2) ? grid : grid / 2;
+  const bool pair = variant == 2 || variant == 3 || variant == 5;
+  const double per_mma = pair ? 2.0 * 256 * 256 * 64 : 2.0 * 128 * 256 * 64;
+  const double issuers = pair ? grid / 2 : grid;
   *tflops_out = (float)(issuers * 4.0 * iters * per_mma / (ms * 1e-3) / 1e12);
   return st;
 }
