@@ -260,11 +260,14 @@ def cpu_baseline(rows_sample: int = 1024, cols_sample: int = 2048, seed: int = 0
     t_total = 0.0
     flops = 0
     seen = {}
-    cache = cache or {}
+    if cache is None:
+        cache = {}
     r, c = rows_sample, cols_sample
     for name, N, K in LAYERS:
         if (N, K) not in seen:
-            d = cache.get((N, K)) or S.llama_linear(N, K, M=M_TOKENS, seed=seed)
+            if (N, K) not in cache:
+                cache[(N, K)] = S.llama_linear(N, K, M=M_TOKENS, seed=seed)
+            d = cache[(N, K)]
             seen[(N, K)] = (S.as_f32(d["X"][:r]), S.as_f32(d["W"][:c]), S.as_f32(d["dY"][:r, :c]))
         X, W, dY = seen[(N, K)]
         T = lambda a: np.ascontiguousarray(a.T)
@@ -402,12 +405,19 @@ def run_ours(args, rank, world, device):
 
 
 def run_reference(args):
-    """The reference arm: the CPU oracle as it stands, on bounded samples."""
+    """The reference arm: the CPU oracle as it stands, on bounded samples.  The
+    token sample of each step shrinks with the number of steps so that the
+    whole run stays within about two and a half minutes (1024 tokens take
+    about 7.5 s on 16 cores)."""
+    f = min(1.0, 20.0 / max(1, args.steps + args.warmup)) ** 0.5   # sample side scale
+    rows = args.ref_rows or max(64, int(1024 * f) // 64 * 64)
+    cols = args.ref_cols or max(128, int(2048 * f) // 128 * 128)
     steps = []
+    cache = {}                    # the synthetic layers are generated once, not per step
     for _ in range(args.warmup):
-        cpu_baseline(args.ref_rows, args.ref_cols)
+        cpu_baseline(rows, cols, args.seed, cache)
     for _ in range(args.steps):
-        steps.append(cpu_baseline(args.ref_rows, args.ref_cols))
+        steps.append(cpu_baseline(rows, cols, args.seed, cache))
     v = statistics.median(s["value"] for s in steps)
     secs = sum(s["seconds"] for s in steps)
     flops_step = sum(6 * M_TOKENS * N * K for _, N, K in LAYERS)
@@ -419,7 +429,7 @@ def run_reference(args):
             "ms_per_step": round(ms, 1), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic (seeded)",
             "config": {"workload": "Llama-7B linear layers fwd+bwd, tokens 32768; each step a "
-                                   f"bounded sample of {args.ref_rows} tokens x {args.ref_cols} "
+                                   f"bounded sample of {rows} tokens x {cols} "
                                    "output features per layer"},
             "cpu_baseline": cb, "seconds_total": round(secs, 1),
             "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -707,8 +717,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ref-rows", type=int, default=1024)
-    ap.add_argument("--ref-cols", type=int, default=2048)
+    ap.add_argument("--ref-rows", type=int, default=None,
+                    help="tokens per layer in each oracle sample (default: 1024 for the "
+                         "cpu_baseline leg; scaled to the step count for --impl reference)")
+    ap.add_argument("--ref-cols", type=int, default=None)
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -741,7 +753,7 @@ def main():
     torch.cuda.set_device(device)
     out, cache = run_ours(args, rank, world, device)
     if rank == 0 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(args.ref_rows, args.ref_cols, args.seed, cache)
+        out["cpu_baseline"] = cpu_baseline(args.ref_rows or 1024, args.ref_cols or 2048, args.seed, cache)
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
