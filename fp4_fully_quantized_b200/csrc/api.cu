@@ -181,7 +181,20 @@ fp4_status fp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
   // Tensor amax of each requested output (NVFP4 only).
   const float* src_row = nullptr;
   const float* src_col = nullptr;
-  if (nv && out) {
+  const bool fused_amax = nv && out && out_t && p->amax_in == nullptr &&
+                          p->amax_in_t == nullptr && p->rht_n == 0 && p->rht_n_t == 16;
+  if (fused_amax) {
+    // plain amax for the row-wise output and the amax of the column-rotated
+    // tensor for the transposed one, from one read of x
+    if (cudaMemsetAsync(out->amax, 0, sizeof(float), s) != cudaSuccess ||
+        cudaMemsetAsync(out_t->amax, 0, sizeof(float), s) != cudaSuccess)
+      return FP4_ERR_CUDA;
+    if (launch_amax_cols_rht(x, rows, cols, ld, 16, mask_t, out_t->amax, out->amax, s) != cudaSuccess)
+      return FP4_ERR_CUDA;
+    src_row = out->amax;
+    src_col = out_t->amax;
+  }
+  if (nv && out && !fused_amax) {
     src_row = p->amax_in;
     if (src_row == nullptr) {
       if (cudaMemsetAsync(out->amax, 0, sizeof(float), s) != cudaSuccess) return FP4_ERR_CUDA;
@@ -190,16 +203,17 @@ fp4_status fp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
       src_row = out->amax;
     }
   }
-  if (nv && out_t) {
+  if (nv && out_t && !fused_amax) {
     src_col = p->amax_in_t;
     if (src_col == nullptr) {
       if (out && p->amax_in == nullptr && p->rht_n == 0 && p->rht_n_t == 0) {
         src_col = out->amax;      // same tensor, same orientation-free amax
       } else {
         if (cudaMemsetAsync(out_t->amax, 0, sizeof(float), s) != cudaSuccess) return FP4_ERR_CUDA;
-        cudaError_t e = p->rht_n_t
-            ? launch_amax_cols(x, rows, cols, ld, p->rht_n_t, mask_t, out_t->amax, s)
-            : launch_amax_rows(x, rows, cols, ld, 0, 0, out_t->amax, s);
+        cudaError_t e = p->rht_n_t == 16
+            ? launch_amax_cols_rht(x, rows, cols, ld, 16, mask_t, out_t->amax, nullptr, s)
+            : p->rht_n_t ? launch_amax_cols(x, rows, cols, ld, p->rht_n_t, mask_t, out_t->amax, s)
+                         : launch_amax_rows(x, rows, cols, ld, 0, 0, out_t->amax, s);
         if (e != cudaSuccess) return FP4_ERR_CUDA;
         src_col = out_t->amax;
       }

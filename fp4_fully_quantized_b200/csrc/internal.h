@@ -41,6 +41,13 @@ cudaError_t launch_amax_rows(const void* x, int64_t rows, int64_t cols, int64_t 
                              int rht_n, uint32_t rht_mask, float* amax, cudaStream_t s);
 cudaError_t launch_amax_cols(const void* x, int64_t rows, int64_t cols, int64_t ld,
                              int rht_n, uint32_t rht_mask, float* amax, cudaStream_t s);
+// Amax of x rotated down its columns (16-row Hadamard blocks; rows must be a
+// multiple of 16; other block sizes return an error) and, when amax_plain is
+// not NULL, the plain amax, from one read.  Both destinations must be zeroed
+// first.
+cudaError_t launch_amax_cols_rht(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                                 int rht_n, uint32_t rht_mask, float* amax_col,
+                                 float* amax_plain, cudaStream_t s);
 cudaError_t launch_quant_rows(const RowQuantArgs& a, cudaStream_t s);
 // Transposed output: the quantized operand is x^T ([cols, rows]); rows of x
 // are the blocked dimension.  Fields keep the meaning of RowQuantArgs with

@@ -154,6 +154,59 @@ amax_plain_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t col
 }
 
 // ---------------------------------------------------------------------------
+// Amax of the column-rotated tensor (the transposed operand's Hadamard runs
+// down x's columns in blocks of RHT_N rows), optionally together with the
+// plain amax, from one read of x.  A warp takes RHT_N rows x 256 columns:
+// lane l loads its 8 columns of every row (RHT_N 16-byte loads in flight),
+// then rotates each of its 8 columns in registers.
+// ---------------------------------------------------------------------------
+template <int RHT_N>
+__global__ void __launch_bounds__(kThreads)
+amax_cols_rht_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+                     uint32_t rht_mask, float* amax_col, float* amax_plain) {
+  const int64_t segs = (cols + 255) / 256, units = (rows / RHT_N) * segs;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const float cn = rht_scale<RHT_N>();
+  float mc = 0.0f, mp = 0.0f;
+  for (int64_t u = warp0; u < units; u += nwarps) {
+    const int64_t rb = u / segs;
+    const int64_t c = (u - rb * segs) * 256 + 8 * lane;
+    if (c >= cols) continue;                  // rows % RHT_N == 0, cols % 8 == 0
+    const __nv_bfloat16* xp = x + rb * RHT_N * ld + c;
+    uint4 raw[RHT_N];
+#pragma unroll
+    for (int q = 0; q < RHT_N; ++q) raw[q] = ld_nc_v4(xp + q * ld);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {             // column c + e
+      float v[RHT_N];
+#pragma unroll
+      for (int q = 0; q < RHT_N; ++q) {
+        const uint32_t w = (&raw[q].x)[e >> 1];
+        v[q] = __uint_as_float((e & 1) ? (w & 0xFFFF0000u) : (w << 16));
+        mp = absmax_keep_nan(mp, v[q]);
+        if ((rht_mask >> q) & 1u) v[q] = -v[q];
+      }
+#pragma unroll
+      for (int hh = 1; hh < RHT_N; hh <<= 1) {
+#pragma unroll
+        for (int q = 0; q < RHT_N; ++q) {
+          if (q & hh) continue;
+          const float a = v[q], b = v[q + hh];
+          v[q] = __fadd_rn(a, b);
+          v[q + hh] = __fsub_rn(a, b);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < RHT_N; ++q) mc = absmax_keep_nan(mc, __fmul_rn(v[q], cn));
+    }
+  }
+  block_amax_atomic(mc, amax_col);
+  if (amax_plain != nullptr) block_amax_atomic(mp, amax_plain);
+}
+
+// ---------------------------------------------------------------------------
 // Row-wise quantization (NVFP4 BS = 16 or MXFP4 BS = 32).  A warp takes one
 // row segment of 32 x kRowChunks 16-byte chunks (1024 elements): lane l owns
 // chunks l, l + 32, ... of the segment, all of whose loads are issued before
@@ -792,6 +845,18 @@ cudaError_t launch_amax_rows(const void* x, int64_t rows, int64_t cols, int64_t 
   if (rht_n == 16) amax_rows_kernel<16><<<grid, kThreads, 0, s>>>(xp, rows, cols, ld, mask, amax);
   else if (rht_n == 32) amax_rows_kernel<32><<<grid, kThreads, 0, s>>>(xp, rows, cols, ld, mask, amax);
   else amax_rows_kernel<0><<<grid, kThreads, 0, s>>>(xp, rows, cols, ld, mask, amax);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_amax_cols_rht(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                                 int rht_n, uint32_t mask, float* amax_col, float* amax_plain,
+                                 cudaStream_t s) {
+  auto xp = static_cast<const __nv_bfloat16*>(x);
+  const int64_t units = (rows / rht_n) * ((cols + 255) / 256);
+  const int grid = grid_for(units, kThreads / 32, 8);
+  if (rht_n != 16) return cudaErrorInvalidValue;   // 16-point blocks only (NVFP4)
+  amax_cols_rht_kernel<16><<<grid, kThreads, 0, s>>>(xp, rows, cols, ld, mask, amax_col, amax_plain);
   count_launches(1);
   return cudaGetLastError();
 }

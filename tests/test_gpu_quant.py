@@ -86,9 +86,12 @@ def test_nvfp4_transposed(gpu_lib, shape, rnd, rht):
     _check_1d(qt, ref, 0)
 
 
-def test_nvfp4_row_and_transposed_together(gpu_lib):
+@pytest.mark.parametrize("shape", [(128, 256), (48, 80), (1024, 4096), (16, 16), (64, 272)])
+def test_nvfp4_row_and_transposed_together(gpu_lib, shape):
+    """Row-wise RTN + transposed SR with a 16-point Hadamard on the transposed
+    operand (the wgrad-RHT layer's X and dY): both amaxes come from one read."""
     F = gpu_lib
-    x, _ = S.outlier_columns(128, 256, seed=0)
+    x, _ = S.outlier_columns(*shape, seed=0)
     q, qt = _gpu_quant(F, x, 0, round=RTN, round_t=SR, rht_n_t=16, seed=0, stream_t=3, col=True)
     xf = S.as_f32(x)
     _check_1d(q, O.nvfp4_quantize_1d(xf), 0)
