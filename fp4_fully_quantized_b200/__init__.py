@@ -34,7 +34,7 @@ EXPORTS = ("fp4_qtensor_sizes", "fp4_qparams_default", "fp4_workspace_bytes", "f
            "fp4_gemm", "fqt_linear_cfg_default", "fqt_linear_fwd", "fqt_linear_bwd",
            "fp4_read_device_status", "fp4_clear_device_status", "fp4_status_str",
            "fp4_abi_version", "fp4_kernel_launches", "fp4_gemm_noalloc", "fp4_mma_rate",
-           "fp4_quant_noise")
+           "fp4_quant_noise", "fp4_gemm_quant")
 
 
 class Fp4Error(RuntimeError):
@@ -112,6 +112,9 @@ def load() -> C.CDLL:
     L.fp4_kernel_launches.argtypes = []
     L.fp4_mma_rate.restype = i32
     L.fp4_mma_rate.argtypes = [i32, i32, C.POINTER(C.c_float), vp, sz, vp]
+    L.fp4_gemm_quant.restype = i32
+    L.fp4_gemm_quant.argtypes = [C.POINTER(QTensorC), C.POINTER(QTensorC), C.c_float, vp,
+                                 C.POINTER(QTensorC), vp, vp, sz, vp]
     L.fp4_quant_noise.restype = i32
     L.fp4_quant_noise.argtypes = [vp, i64, i64, i64, C.POINTER(QTensorC), vp, vp, sz, vp]
     L.fp4_gemm_noalloc.restype = i32
@@ -258,6 +261,17 @@ def mma_rate(variant: int = 0, iters: int = 20000, stream=None) -> float:
     _check(load().fp4_mma_rate(variant, iters, C.byref(out), ws.ptr, ws.nbytes, _stream(stream)),
            "fp4_mma_rate")
     return float(out.value)
+
+
+def fp4_gemm_quant(a: QTensor, b: QTensor, out: QTensor, amax_in: torch.Tensor, alpha: float = 1.0,
+                   c_amax: torch.Tensor | None = None, ws: Workspace | None = None, stream=None):
+    """out = NVFP4 1x16 RTN of (alpha * s_dec(a) * s_dec(b) * a_hat @ b_hat^T), encoded in
+    the GEMM epilogue with the supplied tensor amax (device float32 tensor)."""
+    if ws is None:
+        ws = Workspace(a.rows, b.rows, a.cols, device=amax_in.device)
+    code = load().fp4_gemm_quant(C.byref(a.c), C.byref(b.c), float(alpha), _ptr(amax_in),
+                                 C.byref(out.c), _ptr(c_amax), ws.ptr, ws.nbytes, _stream(stream))
+    _check(code, "fp4_gemm_quant")
 
 
 def fp4_quant_noise(x: torch.Tensor, q: QTensor, sums: torch.Tensor, ws: Workspace | None = None,

@@ -23,10 +23,12 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <cfloat>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
 
+#include "fp4_device.cuh"
 #include "internal.h"
 #include "sm100_ptx.cuh"
 
@@ -56,8 +58,10 @@ struct StParams {
   int M, N, K;
   int atoms_per_rowblk;
   float alpha;
-  void* c; int64_t ldc; int out_f32;
+  void* c; int64_t ldc; int out_mode;     // 0 BF16, 1 FP32, 2 NVFP4 1x16 RTN (q_*)
   float* c_amax;
+  uint8_t* q_codes; uint8_t* q_scales; uint8_t* q_scales_mma;
+  const float* q_amax_in; float* q_amax_out; float* q_s_dec;
   uint32_t* status;
 };
 
@@ -244,8 +248,21 @@ fp4_gemm_sfst_kernel(const __grid_constant__ CUtensorMap tmap_a,
   } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + EPI_WARPS) {
     // ------------------------------------------------------------ epilogue
     const float scale = p.alpha * (*p.a_sdec) * (*p.b_sdec);
-    const int esize = p.out_f32 ? 4 : 2;
+    const int esize = p.out_mode == 1 ? 4 : 2;
     const bool wide_st = (reinterpret_cast<uintptr_t>(p.c) % 32) == 0 && (p.ldc * esize) % 32 == 0;
+    float q_senc = 1.0f;
+    if (p.out_mode == 2) {
+      // encode with the supplied tensor amax (the two-level NVFP4 scale of the
+      // quantizers); record it and the decode scale with the codes
+      const float A = *p.q_amax_in;
+      float q_sdec;
+      fp4dev::nvfp4_global_scales(A, q_senc, q_sdec);
+      if (blockIdx.x == 0 && threadIdx.x == EPI_WARP0 * 32) {
+        if (!(A <= FLT_MAX)) set_status(p.status, FP4_ERR_NONFINITE, 5);
+        *p.q_s_dec = q_sdec;
+        if (p.q_amax_out != p.q_amax_in) *p.q_amax_out = A;
+      }
+    }
     float amax = 0.0f;
     uint32_t tile_iter = 0;
     const int quad = warp & 3, half = (warp - EPI_WARP0) >> 2;
@@ -258,7 +275,7 @@ fp4_gemm_sfst_kernel(const __grid_constant__ CUtensorMap tmap_a,
       const int ncols = min(BN / 2, p.N - nb * BN - c_begin);
       const int64_t col = (int64_t)nb * BN + c_begin;
       const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)c_begin;
-      if (!p.out_f32) {
+      if (p.out_mode == 0) {
         // drain 128 columns in two 64-column loads, packing to BF16 as they
         // arrive (64 registers); two TMEM round trips before the release
         uint32_t pk[64];
@@ -291,6 +308,54 @@ fp4_gemm_sfst_kernel(const __grid_constant__ CUtensorMap tmap_a,
             uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
             for (int q = 0; q < 16; ++q) d4[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          }
+        }
+      } else if (p.out_mode == 2) {
+        // NVFP4 1x16, round to nearest: each 16-column block of the FP32
+        // result gets its E4M3 scale from its own max, then 16 E2M1 codes;
+        // two halves of 64 columns, the accumulator released after the second
+        const int64_t S = p.N >> 4, S4 = (S + 3) & ~3LL;
+#pragma unroll 1
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t v[64];
+          tmem_ld32_nowait(taddr + 64 * h2, v);
+          tmem_ld32_nowait(taddr + 64 * h2 + 32, v + 32);
+          asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+          if (h2 == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);
+          }
+          if (ncols > 0) {
+            uint32_t cw[8];
+            uint32_t sfw = 0;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+              float o[16];
+              float bmax = 0.0f;
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                o[e] = __uint_as_float(v[16 * b + e]) * scale;
+                bmax = fmaxf(bmax, fabsf(o[e]));
+              }
+              amax = fmaxf(amax, bmax);
+              const uint32_t sf = fp4dev::e4m3_rn_sat(__fdiv_rn(__fmul_rn(bmax, q_senc), 6.0f));
+              const float inv = (sf == 0u || sf == 127u)
+                                    ? 0.0f : fminf(__fdiv_rn(q_senc, fp4dev::e4m3_value(sf)), FLT_MAX);
+#pragma unroll
+              for (int e = 0; e < 16; ++e) o[e] = __fmul_rn(o[e], inv);
+              cw[2 * b] = fp4dev::e2m1x8_rn(o);
+              cw[2 * b + 1] = fp4dev::e2m1x8_rn(o + 8);
+              sfw |= sf << (8 * b);
+            }
+            const int64_t c0 = col + 64 * h2;              // first column of these 4 blocks
+            uint4* cd = reinterpret_cast<uint4*>(p.q_codes + row * (p.N >> 1) + (c0 >> 1));
+            cd[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+            cd[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+            const int64_t sb0 = c0 >> 4;                   // a multiple of 4
+            if (p.q_scales != nullptr) *reinterpret_cast<uint32_t*>(p.q_scales + row * S + sb0) = sfw;
+            if (p.q_scales_mma != nullptr)
+              *reinterpret_cast<uint32_t*>(p.q_scales_mma + fp4dev::mma_sf_offset(row, sb0, S4)) = sfw;
           }
         }
       } else {
@@ -388,7 +453,9 @@ fp4_status gemm_launch_sfst(const GemmArgs& g, cudaStream_t s) {
   p.a_sf = g.a_sf; p.b_sf = g.b_sf; p.a_sdec = g.a_sdec; p.b_sdec = g.b_sdec;
   p.M = (int)g.M; p.N = (int)g.N; p.K = (int)g.K;
   p.atoms_per_rowblk = nv ? (int)(g.K / 64) : (int)((((g.K / 32) + 3) / 4 * 4) / 4);
-  p.alpha = g.alpha; p.c = g.c; p.ldc = g.ldc; p.out_f32 = g.out_f32;
+  p.alpha = g.alpha; p.c = g.c; p.ldc = g.ldc; p.out_mode = g.out_mode;
+  p.q_codes = g.q_codes; p.q_scales = g.q_scales; p.q_scales_mma = g.q_scales_mma;
+  p.q_amax_in = g.q_amax_in; p.q_amax_out = g.q_amax_out; p.q_s_dec = g.q_s_dec;
   p.c_amax = g.c_amax; p.status = g.status;
   const int tiles = (int)(g.M / BM) * (int)((g.N + BN - 1) / BN);
   const int grid = tiles < sm_count() ? tiles : sm_count();

@@ -86,8 +86,11 @@ struct GemmArgs {
   int64_t M, N, K;
   int fmt;               // FP4_NVFP4 / FP4_MXFP4
   float alpha;
-  void* c; int64_t ldc; int out_f32;
+  void* c; int64_t ldc; int out_mode;    // 0 BF16, 1 FP32, 2 NVFP4 1x16 RTN into q_*
   float* c_amax;
+  // out_mode 2: the quantized output [M, N] and the supplied tensor amax
+  uint8_t* q_codes; uint8_t* q_scales; uint8_t* q_scales_mma;
+  const float* q_amax_in; float* q_amax_out; float* q_s_dec;
   uint32_t* status;
 };
 fp4_status gemm_launch(const GemmArgs& g, cudaStream_t s);

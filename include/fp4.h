@@ -176,6 +176,23 @@ fp4_status fp4_gemm(const fp4_qtensor* a, const fp4_qtensor* b, float alpha, voi
                     int64_t ldc, int32_t out_dtype, float* c_amax, void* ws,
                     size_t ws_bytes, void* stream);
 
+/* The same GEMM with the result quantized in the epilogue instead of
+ * written as BF16/FP32: each FP32 value C[m, n] (as fp4_gemm computes it)
+ * is encoded to NVFP4 1x16 with round-to-nearest, exactly as fp4_quantize
+ * encodes a row-wise output with a supplied tensor amax, into `out`
+ * (rows M, cols N, FP4_NVFP4, FP4_BLOCK_1D; codes and scales_mma required,
+ * logical scales optional; out->amax receives *out_amax_in and out->s_dec the
+ * matching decode scale).  The tensor amax must be supplied (device float:
+ * for example the previous step's c_amax of this output, "delayed
+ * scaling"); c_amax (nullable) receives this call's max |C| for the next
+ * one.  The output is never stored in BF16: it replaces a BF16 write and the
+ * quantizer's two reads of it ("FP4 All the Way" / "Quartet" pages: quantize
+ * operands in fused kernels).  Shape and alignment rules as fp4_gemm, plus
+ * out->codes 16-byte and the scale pointers 4-byte aligned. */
+fp4_status fp4_gemm_quant(const fp4_qtensor* a, const fp4_qtensor* b, float alpha,
+                          const float* out_amax_in, fp4_qtensor* out, float* c_amax, void* ws,
+                          size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------------- */
 /* Linear layer  Y = X W^T  with X [M, K], W [N, K], dY [M, N]:            */
 /*   fprop  Y  = X . W^T      (contract K)                                 */
