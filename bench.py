@@ -649,7 +649,10 @@ def run_case(args, device):
     """A single kernel family on one small problem (for profiler captures):
     --case gemm: NVFP4 fprop-style GEMM [m, k] x [n, k]^T, BF16 out;
     --case quant: NVFP4 row-wise RTN + transposed SR of a [m, k] tensor;
-    --case quant_sr: both outputs stochastically rounded (the dY quantization)."""
+    --case quant_sr: both outputs stochastically rounded (the dY quantization);
+    --case gemm_quant / gemm_then_quant: the GEMM with its result encoded to
+    NVFP4 in the epilogue, against the GEMM's BF16 output quantized afterwards
+    (both with a supplied output amax)."""
     import fp4_fully_quantized_b200 as F
     import fqt_synth as S
     F.load()
@@ -676,7 +679,14 @@ def run_case(args, device):
         F.fp4_quantize(x, qa, ws=ws)
         F.fp4_quantize(w, qb, qbt, block=F.BLOCK_2D, ws=ws)
         y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
-        fn = lambda: F.fp4_gemm(qa, qb, y, ws=ws)
+        qy = F.QTensor.empty(M, N, device=device, logical_scales=False)
+        y_amax = torch.ones(1, dtype=torch.float32, device=device)   # supplied (delayed) amax
+        if args.case == "gemm_quant":          # result encoded to NVFP4 in the epilogue
+            fn = lambda: F.fp4_gemm_quant(qa, qb, qy, y_amax, ws=ws)
+        elif args.case == "gemm_then_quant":   # BF16 result, then the quantizer
+            fn = lambda: (F.fp4_gemm(qa, qb, y, ws=ws), F.fp4_quantize(y, qy, amax_in=y_amax, ws=ws))
+        else:
+            fn = lambda: F.fp4_gemm(qa, qb, y, ws=ws)
         units, unit = 2 * M * N * K / 1e12, "TFLOP/s"
     for _ in range(args.warmup):
         fn()
@@ -695,7 +705,8 @@ def run_case(args, device):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--case", choices=["gemm", "quant", "quant_sr", "sweep", "swiglu"], default=None,
+    ap.add_argument("--case", choices=["gemm", "gemm_quant", "gemm_then_quant", "quant", "quant_sr",
+                                       "sweep", "swiglu"], default=None,
                     help="time one kernel family on one problem (profiling), or the "
                          "quantizer sweep over 2^n elements")
     ap.add_argument("--rounds", default=None,
