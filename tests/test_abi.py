@@ -93,3 +93,38 @@ def test_argument_errors_return_before_launch(lib):
     cfg = F.linear_cfg(F.NVFP4, rht_mask=F.RHT_FPROP)
     assert lib.fqt_linear_fwd(C.byref(cfg), 128, 128, 128, fake_x, fake_x, fake_x,
                               C.byref(F.SavedC()), ws, 256, None) == 9
+
+
+def test_gemm_quant_and_noise_argument_errors(lib):
+    """The epilogue-quantized GEMM and the noise diagnostic validate on the
+    host and return before any launch."""
+    a, b = _q(128, 128), _q(256, 128)
+    out = _q(128, 256)
+    amax = C.c_void_p(1 << 23)
+    ws = C.c_void_p(1 << 21)
+    # missing supplied amax / output
+    assert lib.fp4_gemm_quant(C.byref(a), C.byref(b), 1.0, None, C.byref(out), None, ws, 256,
+                              None) == 1
+    assert lib.fp4_gemm_quant(C.byref(a), C.byref(b), 1.0, amax, None, None, ws, 256, None) == 1
+    # output must be NVFP4 1x16 of shape [M, N]
+    assert lib.fp4_gemm_quant(C.byref(a), C.byref(b), 1.0, amax, C.byref(_q(128, 256, 1)), None,
+                              ws, 256, None) == 4
+    assert lib.fp4_gemm_quant(C.byref(a), C.byref(b), 1.0, amax, C.byref(_q(128, 256, 0, 1)), None,
+                              ws, 256, None) == 4
+    assert lib.fp4_gemm_quant(C.byref(a), C.byref(b), 1.0, amax, C.byref(_q(256, 256)), None,
+                              ws, 256, None) == 2
+    # GEMM shape rules still apply
+    assert lib.fp4_gemm_quant(C.byref(_q(96, 128)), C.byref(b), 1.0, amax, C.byref(_q(96, 256)),
+                              None, ws, 256, None) == 2
+    # workspace
+    assert lib.fp4_gemm_quant(C.byref(a), C.byref(b), 1.0, amax, C.byref(out), None, None, 0,
+                              None) == 5
+    # noise diagnostic: null sums, shape mismatch, misaligned sums, bad format
+    x = C.c_void_p(1 << 20)
+    q = _q(32, 64)
+    sums = C.c_void_p(1 << 24)
+    assert lib.fp4_quant_noise(x, 32, 64, 64, C.byref(q), None, None, 0, None) == 1
+    assert lib.fp4_quant_noise(x, 32, 128, 128, C.byref(q), sums, None, 0, None) == 2
+    assert lib.fp4_quant_noise(x, 32, 64, 64, C.byref(q), C.c_void_p((1 << 24) + 4), None, 0,
+                               None) == 3
+    assert lib.fp4_quant_noise(x, 32, 64, 64, C.byref(_q(32, 64, 5)), sums, None, 0, None) == 4
