@@ -172,9 +172,31 @@ def qparams_for(cfg, which):
                 sr_seed=cfg.seed, sr_stream=1, sr_stream_t=2)
 
 
-def plan(F, layers, ws):
+class DwAllReduce:
+    """Data-parallel gradient exchange: each layer's FP32 dW [N, K] summed over
+    all ranks.  It is issued right after that layer's wgrad; NCCL runs it on
+    its own stream, after the work already queued, so it overlaps the next
+    layer's kernels.  `finish` makes the launching stream wait for every
+    pending sum; every rank issues the same sums in the same order."""
+
+    def __init__(self, world: int):
+        self.world, self.works = world, []
+
+    def issue(self, dw: torch.Tensor) -> None:
+        if self.world > 1:
+            self.works.append(torch.distributed.all_reduce(dw, async_op=True))
+
+    def finish(self) -> None:
+        for w in self.works:
+            w.wait()
+        self.works.clear()
+
+
+def plan(F, layers, ws, dp=None):
     """The calls of one step: (kind, units, thunk, label) -- the calls
-    fqt_linear_fwd / fqt_linear_bwd make for each layer."""
+    fqt_linear_fwd / fqt_linear_bwd make for each layer, and with `dp` (a
+    DwAllReduce) the dW sum after each wgrad and the wait for all of them at
+    the end of the step."""
     calls = []
     for L in layers:
         sv = L.sv
@@ -194,6 +216,10 @@ def plan(F, layers, ws):
             ("gemm", 2 * L.M * L.N * L.K, lambda L=L, sv=sv: F.fp4_gemm(sv.dyq_t, sv.xq_t, L.dw, ws=ws),
              f"wgrad {tag}"),
         ]
+        if dp is not None:
+            calls.append(("comm", L.N * L.K * 4, lambda L=L: dp.issue(L.dw), f"dW all-reduce {tag}"))
+    if dp is not None:
+        calls.append(("comm", 0, dp.finish, "dW all-reduce wait"))
     return calls
 
 
@@ -208,9 +234,10 @@ def step(calls, events=None):
             fn()
 
 
-def e2e_run(F, layers, cache, cfg, ws, steps, device):
+def e2e_run(F, layers, cache, cfg, ws, steps, device, dp=None):
     """Same workload through fqt_linear_fwd / fqt_linear_bwd with HOST buffers:
-    every step copies X, W, dY in from pinned memory and Y, dX, dW out."""
+    every step copies X, W, dY in from pinned memory and Y, dX, dW out (dW
+    after its sum over ranks when `dp` is given)."""
     host = {}
     for (N, K), src in cache.items():
         host[(N, K)] = {
@@ -229,9 +256,16 @@ def e2e_run(F, layers, cache, cfg, ws, steps, device):
             L.dy.copy_(h["dY"], non_blocking=True)
             F.fqt_linear_fwd(L.cfg, L.x, L.w, L.y, L.sv, ws)
             F.fqt_linear_bwd(L.cfg, L.dy, L.sv, L.dx, L.dw, ws)
+            if dp is not None:
+                dp.issue(L.dw)
             h["Y"].copy_(L.y, non_blocking=True)
             h["dX"].copy_(L.dx, non_blocking=True)
-            h["dW"].copy_(L.dw, non_blocking=True)
+            if dp is None:
+                h["dW"].copy_(L.dw, non_blocking=True)
+        if dp is not None:
+            dp.finish()
+            for L in layers:
+                host[(L.N, L.K)]["dW"].copy_(L.dw, non_blocking=True)
 
     one()
     torch.cuda.synchronize()
@@ -299,7 +333,8 @@ def run_ours(args, rank, world, device):
         cfg.rht_mask = F.RHT_WGRAD
     layers, cache = make_layers(F, cfg, device, args.seed + rank)
     ws = F.Workspace(device=device)
-    calls = plan(F, layers, ws)
+    dp = DwAllReduce(world) if args.dp_allreduce else None
+    calls = plan(F, layers, ws, dp)
     clk = ClockSampler(device.index).__enter__()     # sampling before the timed region
     for _ in range(args.warmup):
         step(calls)
@@ -334,6 +369,8 @@ def run_ours(args, rank, world, device):
     breakdown = {}
     for per in evs:
         for (kind, units, _f, label), (a, b) in zip(calls, per):
+            if kind == "comm":          # enqueue only; the sum runs on NCCL's stream
+                continue
             d = breakdown.setdefault(label, [kind, units, 0.0, 0])
             d[2] += a.elapsed_time(b)
             d[3] += 1
@@ -359,7 +396,7 @@ def run_ours(args, rank, world, device):
 
     e2e = None
     if not args.no_e2e:
-        e_ms, h2d, d2h = e2e_run(F, layers, cache, cfg, ws, args.e2e_steps, device)
+        e_ms, h2d, d2h = e2e_run(F, layers, cache, cfg, ws, args.e2e_steps, device, dp)
         e_max = max_over_ranks(e_ms, device, world)
         e2e = {"value": round(whole_job_rate(flops_step, world, e_max) / 1e12, 2),
                "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -382,7 +419,9 @@ def run_ours(args, rank, world, device):
                    "format": args.fmt, "rounding": "RTN fwd, SR bwd/update" if fmt == F.NVFP4
                    else "RTN fwd/bwd", "weights": "16x16 tiles" if fmt == F.NVFP4 else "1x32",
                    "rht": {0: "off", 4: "wgrad 16-pt", 7: "all GEMMs 32-pt"}.get(cfg.rht_mask),
-                   "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}"},
+                   "l2": "inputs larger than L2 (no flush)",
+                   "parallelism": f"dp x{world}, dW all-reduce (NCCL, overlapped)"
+                   if dp is not None else f"replicas x{world}"},
         "roofline": {"kernel": "fp4_gemm_sfst_kernel (tcgen05 block-scaled, scales staged by tcgen05.st)", "bound": "tensor",
                      "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1),
                      "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4),
@@ -724,6 +763,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--fmt", choices=["nvfp4", "mxfp4"], default="nvfp4")
     ap.add_argument("--wgrad-rht", action="store_true")
+    ap.add_argument("--dp-allreduce", action="store_true",
+                    help="data parallel: sum each layer's dW over the ranks (NCCL) inside the step")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2)
