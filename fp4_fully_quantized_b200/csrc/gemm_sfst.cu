@@ -1,8 +1,8 @@
 // gemm_sfst.cu -- block-scaled FP4 GEMM with scale factors staged by
 // tcgen05.st (one SM per 128 x 256 output tile).
 //
-// Same product as gemm_sm100.cu ("FP4" page, How it works: FP4 tensor-core
-// products with higher-precision accumulation).  The difference is how the
+// The product is the one of the "FP4" page (How it works: FP4 tensor-core
+// products with higher-precision accumulation).  The design point is how the
 // per-block scales reach tensor memory.  Copying them with tcgen05.cp from the
 // MMA-issuing thread puts 12 copies per 256-element K step into the same
 // in-order tensor pipe as the 4 MMAs, and measured on B200 the MMAs then run at

@@ -79,7 +79,7 @@ struct Quant2DArgs {
 };
 cudaError_t launch_quant_2d(const Quant2DArgs& a, cudaStream_t s);
 
-// --- GEMM (gemm_sm100.cu) -------------------------------------------------
+// --- GEMM (gemm.cu -> gemm_sfst.cu) ---------------------------------------
 struct GemmArgs {
   const uint8_t* a_codes; const uint8_t* a_sf; const float* a_sdec;
   const uint8_t* b_codes; const uint8_t* b_sf; const float* b_sdec;

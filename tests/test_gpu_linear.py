@@ -128,3 +128,107 @@ def test_linear_quantized_result_tracks_unquantized(gpu_lib):
     assert rel_fro(y, X @ W.T) < 0.2
     assert rel_fro(dx, dY @ W) < 0.3
     assert rel_fro(dw, dY.T @ X) < 0.3
+
+
+# BF16 outputs: the FP32-accumulation bar plus at most 2^-9 relative rounding
+# per element from the final BF16 store.
+TOL_BF16 = TOL + 2.0 ** -9
+
+
+@pytest.mark.parametrize("variant", ["nvfp4", "mxfp4"])
+def test_llama_qkvo_layer_full_size_sampled(gpu_lib, variant):
+    """One 7B QKVO layer (M = 32768 tokens, N = K = 4096) through
+    fqt_linear_fwd / fqt_linear_bwd in the configuration the step benchmark
+    times (BF16 Y and dX, FP32 dW).  The oracle checks W, W^T and X^T in full,
+    32 sampled rows of X, dY and dY^T (with the full-tensor amax), and 32
+    sampled rows of Y, dX and dW over the full contraction."""
+    F = gpu_lib
+    M, N, K = 32768, 4096, 4096
+    nv = variant == "nvfp4"
+    fmt, bs = (0, 16) if nv else (1, 32)
+    d = S.llama_linear(N, K, M=M, seed=0)
+    cfg = F.linear_cfg(fmt, out_dtype=F.OUT_BF16, seed=0)
+    sv = F.Saved.empty(M, N, K, cfg, logical_scales=False)
+    ws = F.Workspace(M, N, K)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    dx = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    dw = torch.empty((N, K), dtype=torch.float32, device="cuda")
+    F.fqt_linear_fwd(cfg, d["X"].cuda(), d["W"].cuda(), y, sv, ws)
+    F.fqt_linear_bwd(cfg, d["dY"].cuda(), sv, dx, dw, ws)
+    torch.cuda.synchronize()
+    assert ws.status() == 0
+
+    X, W, dY = (S.as_f32(d[k]) for k in ("X", "W", "dY"))
+    T = lambda a: np.ascontiguousarray(a.T)
+    rn, m = cfg.rht_n, cfg.rht_mask
+    rnd = lambda r: "sr" if r == 1 else "rtn"
+    Ax, Ady = O.amax(X), O.amax(dY)
+
+    def q1(a, r, rht, stream, amax_in=None, row_offset=0):
+        if nv:
+            return O.nvfp4_quantize_1d(a, rnd(r), rht_n=rht, rht_seed=0, sr_seed=0,
+                                       sr_stream=stream, amax_in=amax_in, row_offset=row_offset)
+        return O.mxfp4_quantize(a, rnd(r), rht_n=rht, rht_seed=0, sr_seed=0, sr_stream=stream,
+                                row_offset=row_offset)
+
+    def deq(q, blk=(1, 16)):
+        return O.dequantize(q["codes"], q["scales"], blk if nv else (1, 32), not nv)
+
+    def sel_rows(q, idx):
+        return {"codes": q["codes"][idx], "scales": q["scales"][idx], "s_dec": q["s_dec"]}
+
+    def got_codes(t, idx=None):
+        c = t.codes.cpu().numpy().reshape(t.rows, t.cols // 2)
+        return c if idx is None else c[idx]
+
+    def got_scales(t):
+        return from_mma_layout(t.scales_mma.cpu().numpy(), t.rows, t.cols // bs)
+
+    def sampled(a, idx, r, rht, stream, A):
+        """Rows idx of the quantization of a, one oracle call per row."""
+        parts = [q1(a[i:i + 1], r, rht, stream, A, int(i)) for i in idx]
+        return {"codes": np.concatenate([p["codes"] for p in parts]),
+                "scales": np.concatenate([p["scales"] for p in parts]),
+                "s_dec": parts[0]["s_dec"]}
+
+    rng = np.random.default_rng(11)
+    rows = np.sort(rng.choice(M, 32, replace=False))
+    nsel = np.sort(rng.choice(N, 32, replace=False))
+
+    # weights and X^T in full
+    if nv:
+        wq, wq_t, wblk = O.nvfp4_quantize_2d(W), O.nvfp4_quantize_2d(T(W)), (16, 16)
+    else:
+        wq = q1(W, cfg.round_fwd, rn if m & 1 else 0, 0)
+        wq_t = q1(T(W), cfg.round_fwd, rn if m & 2 else 0, 0)
+        wblk = (1, 32)
+    xq_t = q1(T(X), cfg.round_x_t, rn if m & 4 else 0, 3)
+    for name, t, ref in (("wq", sv.wq, wq), ("wq_t", sv.wq_t, wq_t), ("xq_t", sv.xq_t, xq_t)):
+        assert np.array_equal(got_codes(t), ref["codes"]), name
+        sc = expand_2d(ref["scales"], t.rows) if t.block == 1 else ref["scales"]
+        assert np.array_equal(got_scales(t), sc), name
+        assert float(t.s_dec.item()) == float(ref["s_dec"]), name
+
+    # sampled rows of X, dY (row-wise) and dY^T
+    xq = sampled(X, rows, cfg.round_fwd, rn if m & 1 else 0, 0, Ax)
+    dyq = sampled(dY, rows, cfg.round_bwd, rn if m & 2 else 0, 1, Ady)
+    dYt = T(dY[:, nsel])                                   # rows n of dY^T
+    parts = [q1(dYt[j:j + 1], cfg.round_bwd, rn if m & 4 else 0, 2, Ady, int(n))
+             for j, n in enumerate(nsel)]
+    dyq_t = {"codes": np.concatenate([p["codes"] for p in parts]),
+             "scales": np.concatenate([p["scales"] for p in parts]), "s_dec": parts[0]["s_dec"]}
+    for name, t, ref, idx in (("xq", sv.xq, xq, rows), ("dyq", sv.dyq, dyq, rows),
+                              ("dyq_t", sv.dyq_t, dyq_t, nsel)):
+        assert np.array_equal(got_codes(t, idx), ref["codes"]), name
+        assert np.array_equal(got_scales(t)[idx], ref["scales"]), name
+        assert float(t.s_dec.item()) == float(ref["s_dec"]), name
+
+    # outputs over the full contraction
+    sd = lambda q: float(q["s_dec"])
+    ry = O.gemm(deq(xq), deq(wq, wblk), s_dec_a=sd(xq), s_dec_b=sd(wq))
+    rdx = O.gemm(deq(dyq), deq(wq_t, wblk), s_dec_a=sd(dyq), s_dec_b=sd(wq_t))
+    rdw = O.gemm(deq(dyq_t), deq(xq_t), s_dec_a=sd(dyq_t), s_dec_b=sd(xq_t))
+    ri, ni = torch.from_numpy(rows).cuda(), torch.from_numpy(nsel).cuda()
+    assert rel_fro(y[ri].float().cpu().numpy(), ry) <= TOL_BF16
+    assert rel_fro(dx[ri].float().cpu().numpy(), rdx) <= TOL_BF16
+    assert rel_fro(dw[ni].cpu().numpy(), rdw) <= TOL
