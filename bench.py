@@ -39,9 +39,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 FP4_PER_BF16 = 4.0          # nominal dense FP4 / dense BF16 tensor throughput (9 / 2.25 PF)
 # DRAM bytes (read + write) per GEMM launch, averaged over the 21 GEMM
 # launches of one step: ncu dram__bytes_read.sum + dram__bytes_write.sum
-# (single pass) of fp4_gemm_sfst_kernel as it stands, 344.9 MB read + 249.0 MB
+# (single pass) of fp4_gemm_sfst_kernel as it stands, 345.3 MB read + 249.2 MB
 # written.  Set to None whenever the GEMM kernel changes until re-measured.
-GEMM_DRAM_BYTES_PER_LAUNCH = 5.939e8
+GEMM_DRAM_BYTES_PER_LAUNCH = 5.945e8
 # Algorithmic bytes per element of one quantize call producing row-wise and
 # transposed outputs with an in-kernel amax: amax read 2 B + encode read 2 B
 # + two outputs of (0.5 B codes + 1/16 B scales).
