@@ -5,9 +5,9 @@ the backward and update passes) is pinned by what the definition of an
 unbiased stochastic rounding fixes: lattice points are fixed, the rounding
 is unbiased (mean over 4096 seeds within 3 sigma), the up-probability is the
 exact fraction of the gap, and for a fixed draw the result is monotone in v.
-Philox is pinned statistically (uniformity, bit balance, independence of
-streams) and by its counter structure; exact agreement with the published
-known-answer vectors is not checked offline (parity unpinned beyond that).
+Philox is pinned block for block against an independent Philox4x32-10
+(cuRAND's host generator, which runs on the CPU), statistically (uniformity,
+bit balance, independence of streams) and by its counter structure.
 """
 import numpy as np
 
@@ -106,3 +106,73 @@ def test_philox_uniformity_and_bit_balance():
     x = d.astype(np.float64) / 2**32 - 0.5
     r = np.corrcoef(x[:-1], x[1:])[0, 1]
     assert abs(r) < 5 / np.sqrt(n)
+
+
+# --- known answers from an independent Philox4x32-10: cuRAND's host generator
+def _curand():
+    """cuRAND (CUDA toolkit or the nvidia-curand wheel), or None."""
+    import ctypes
+    import glob
+    import os
+    cands = []
+    for root in (os.environ.get("CUDA_HOME", ""), "/usr/local/cuda"):
+        if root:
+            cands += sorted(glob.glob(os.path.join(root, "lib64", "libcurand.so*")))
+    try:
+        import nvidia.curand
+        cands += sorted(glob.glob(os.path.join(nvidia.curand.__path__[0], "lib", "libcurand.so*")))
+    except ImportError:
+        pass
+    for c in cands:
+        try:
+            return ctypes.CDLL(c)
+        except OSError:
+            continue
+    return None
+
+
+def _curand_philox_blocks(seed: int, n_blocks: int):
+    """n_blocks 4-word outputs of cuRAND's host CURAND_RNG_PSEUDO_PHILOX4_32_10
+    generator for `seed` (runs on the CPU; no GPU needed)."""
+    import ctypes as C
+    import pytest
+    cr = _curand()
+    if cr is None:
+        pytest.skip("libcurand not found")
+    gen = C.c_void_p()
+    if cr.curandCreateGeneratorHost(C.byref(gen), 161) != 0:   # PHILOX4_32_10
+        pytest.skip("cuRAND host generator unavailable")
+    try:
+        assert cr.curandSetPseudoRandomGeneratorSeed(gen, C.c_ulonglong(seed)) == 0
+        buf = np.empty(4 * n_blocks, np.uint32)
+        assert cr.curandGenerate(gen, buf.ctypes.data_as(C.c_void_p), C.c_size_t(buf.size)) == 0
+    finally:
+        cr.curandDestroyGenerator(gen)
+    return buf.reshape(-1, 4)
+
+
+def test_philox_matches_curand_host_generator():
+    """cuRAND's Philox4x32-10 keys the generator with the 64-bit seed (low
+    word first) and lays its output out as S parallel subsequences: output
+    block c * S + s is the Philox block of counter (c, 0, s, 0).  The oracle's
+    draw i of stream s is word i mod 4 of counter (i / 4, 0, s, 0), so both
+    must agree block for block wherever the layouts meet.  A wrong round
+    count, multiplier, Weyl constant, word order or key schedule in the
+    oracle breaks the agreement everywhere."""
+    for seed in (0, 0x0123456789ABCDEF, 2**64 - 1):
+        blocks = _curand_philox_blocks(seed, 3 * 65536)
+        key = [seed & 0xFFFFFFFF, seed >> 32]
+        # the very first block is counter 0 of subsequence 0
+        assert np.array_equal(blocks[0], O.philox4x32_10([0, 0, 0, 0], key))
+        # the layout's width S: where counter 1 of subsequence 0 sits
+        hit = np.where((blocks == O.philox4x32_10([1, 0, 0, 0], key)).all(axis=1))[0]
+        assert hit.size == 1
+        S = int(hit[0])
+        assert S > 0 and blocks.shape[0] >= 2 * S
+        rng = np.random.default_rng(seed & 0xFFFF)
+        for s in list(rng.integers(0, S, 24)) + [0, 1, 2, 3, S - 1]:
+            for c in (0, 1):
+                want = blocks[c * S + int(s)]
+                assert np.array_equal(O.philox4x32_10([c, 0, int(s), 0], key), want), (seed, c, s)
+                # the oracle's draws of stream s, elements 4c .. 4c + 3
+                assert np.array_equal(O.draws(seed, int(s), 4 * c, 4), want), (seed, c, s)
