@@ -5,7 +5,7 @@
 // The linear-layer entry points compose fp4_quantize and fp4_gemm in the
 // order of a fully quantized linear layer: "FP4 All the Way", Key points
 // (round-to-nearest forward, stochastic rounding in backward and update)
-// and "Quartet", abstract line (fprop, dgrad and wgrad all in FP4).
+// and "Quartet", Abstract (fprop, dgrad and wgrad all in FP4).
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -115,9 +115,11 @@ size_t fp4_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   return sizeof(DeviceStatus);
 }
 
-fp4_status fp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
-                        const fp4_qparams* p, fp4_qtensor* out, fp4_qtensor* out_t, void* ws,
-                        size_t ws_bytes, void* stream) {
+// fp4_quantize; with `dry` it only validates the arguments and returns at the
+// point where the first copy or kernel would be enqueued.
+static fp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                                const fp4_qparams* p, fp4_qtensor* out, fp4_qtensor* out_t,
+                                void* ws, size_t ws_bytes, void* stream, bool dry) {
   if (p == nullptr) return FP4_ERR_NULL;
   if (out == nullptr && out_t == nullptr) return FP4_ERR_NULL;
   if (ws != nullptr && ws_bytes < sizeof(DeviceStatus)) return FP4_ERR_WORKSPACE;
@@ -143,6 +145,7 @@ fp4_status fp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
     fp4_status st;
     if (out && (st = check_qtensor(out, rows, cols, FP4_NVFP4, FP4_BLOCK_2D)) != FP4_OK) return st;
     if (out_t && (st = check_qtensor(out_t, cols, rows, FP4_NVFP4, FP4_BLOCK_2D)) != FP4_OK) return st;
+    if (dry) return FP4_OK;
     float* amax_dst = out ? out->amax : out_t->amax;
     const float* src = p->amax_in;
     if (src == nullptr) {
@@ -174,6 +177,7 @@ fp4_status fp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
     if (p->rht_n_t && rows % p->rht_n_t) return FP4_ERR_SHAPE;
     if ((st = check_qtensor(out_t, cols, rows, p->fmt, FP4_BLOCK_1D)) != FP4_OK) return st;
   }
+  if (dry) return FP4_OK;
   const uint32_t mask = p->rht_n ? fp4dev::rht_sign_mask(p->rht_seed, p->rht_n) : 0u;
   const uint32_t mask_t = p->rht_n_t ? fp4dev::rht_sign_mask(p->rht_seed, p->rht_n_t) : 0u;
   const bool nv = p->fmt == FP4_NVFP4;
@@ -264,8 +268,16 @@ fp4_status fp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
   return FP4_OK;
 }
 
-fp4_status fp4_gemm(const fp4_qtensor* a, const fp4_qtensor* b, float alpha, void* c, int64_t ldc,
-                    int32_t out_dtype, float* c_amax, void* ws, size_t ws_bytes, void* stream) {
+fp4_status fp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                        const fp4_qparams* p, fp4_qtensor* out, fp4_qtensor* out_t, void* ws,
+                        size_t ws_bytes, void* stream) {
+  return quantize_impl(x, rows, cols, ld, p, out, out_t, ws, ws_bytes, stream, false);
+}
+
+// fp4_gemm; with `dry` it only validates the arguments.
+static fp4_status gemm_impl(const fp4_qtensor* a, const fp4_qtensor* b, float alpha, void* c,
+                            int64_t ldc, int32_t out_dtype, float* c_amax, void* ws,
+                            size_t ws_bytes, void* stream, bool dry) {
   if (a == nullptr || b == nullptr || c == nullptr) return FP4_ERR_NULL;
   if (a->codes == nullptr || b->codes == nullptr || a->scales_mma == nullptr ||
       b->scales_mma == nullptr || a->s_dec == nullptr || b->s_dec == nullptr)
@@ -282,6 +294,7 @@ fp4_status fp4_gemm(const fp4_qtensor* a, const fp4_qtensor* b, float alpha, voi
       !aligned16(b->scales_mma))
     return FP4_ERR_ALIGN;
   if (ws == nullptr || ws_bytes < fp4_workspace_bytes(M, N, K)) return FP4_ERR_WORKSPACE;
+  if (dry) return FP4_OK;
   GemmArgs g{};
   g.a_codes = a->codes; g.a_sf = a->scales_mma; g.a_sdec = a->s_dec;
   g.b_codes = b->codes; g.b_sf = b->scales_mma; g.b_sdec = b->s_dec;
@@ -289,6 +302,11 @@ fp4_status fp4_gemm(const fp4_qtensor* a, const fp4_qtensor* b, float alpha, voi
   g.c = c; g.ldc = ldc; g.out_mode = out_dtype == FP4_OUT_F32 ? 1 : 0;
   g.c_amax = c_amax; g.status = status_ptr(ws);
   return gemm_launch(g, as_stream(stream));
+}
+
+fp4_status fp4_gemm(const fp4_qtensor* a, const fp4_qtensor* b, float alpha, void* c, int64_t ldc,
+                    int32_t out_dtype, float* c_amax, void* ws, size_t ws_bytes, void* stream) {
+  return gemm_impl(a, b, alpha, c, ldc, out_dtype, c_amax, ws, ws_bytes, stream, false);
 }
 
 fp4_status fp4_gemm_quant(const fp4_qtensor* a, const fp4_qtensor* b, float alpha,
@@ -356,6 +374,9 @@ static fp4_status check_cfg(const fqt_linear_cfg* cfg) {
   return FP4_OK;
 }
 
+// The layer's calls, run twice: first validating only (`dry`), so that an
+// argument error of any of them returns before anything is enqueued, then
+// for real.
 fp4_status fqt_linear_fwd(const fqt_linear_cfg* cfg, int64_t M, int64_t N, int64_t K,
                           const void* x, const void* w, void* y, fqt_saved* sv, void* ws,
                           size_t ws_bytes, void* stream) {
@@ -375,8 +396,6 @@ fp4_status fqt_linear_fwd(const fqt_linear_cfg* cfg, int64_t M, int64_t N, int64
   px.sr_seed = cfg->seed;
   px.sr_stream = 0;
   px.sr_stream_t = 3;
-  st = fp4_quantize(x, M, K, K, &px, &sv->xq, &sv->xq_t, ws, ws_bytes, stream);
-  if (st != FP4_OK) return st;
   // W: fprop operand [N, K] and dgrad operand W^T [K, N]
   fp4_qparams pw;
   fp4_qparams_default(&pw);
@@ -387,9 +406,16 @@ fp4_status fqt_linear_fwd(const fqt_linear_cfg* cfg, int64_t M, int64_t N, int64
   pw.rht_n = (cfg->rht_mask & FQT_RHT_FPROP) ? rn : 0;
   pw.rht_n_t = (cfg->rht_mask & FQT_RHT_DGRAD) ? rn : 0;
   pw.rht_seed = cfg->seed;
-  st = fp4_quantize(w, N, K, K, &pw, &sv->wq, &sv->wq_t, ws, ws_bytes, stream);
-  if (st != FP4_OK) return st;
-  return fp4_gemm(&sv->xq, &sv->wq, 1.0f, y, N, cfg->out_dtype, nullptr, ws, ws_bytes, stream);
+  for (const bool dry : {true, false}) {
+    st = quantize_impl(x, M, K, K, &px, &sv->xq, &sv->xq_t, ws, ws_bytes, stream, dry);
+    if (st != FP4_OK) return st;
+    st = quantize_impl(w, N, K, K, &pw, &sv->wq, &sv->wq_t, ws, ws_bytes, stream, dry);
+    if (st != FP4_OK) return st;
+    st = gemm_impl(&sv->xq, &sv->wq, 1.0f, y, N, cfg->out_dtype, nullptr, ws, ws_bytes, stream,
+                   dry);
+    if (st != FP4_OK) return st;
+  }
+  return FP4_OK;
 }
 
 fp4_status fqt_linear_bwd(const fqt_linear_cfg* cfg, int64_t M, int64_t N, int64_t K,
@@ -410,11 +436,17 @@ fp4_status fqt_linear_bwd(const fqt_linear_cfg* cfg, int64_t M, int64_t N, int64
   pd.sr_seed = cfg->seed;
   pd.sr_stream = 1;
   pd.sr_stream_t = 2;
-  st = fp4_quantize(dy, M, N, N, &pd, &sv->dyq, &sv->dyq_t, ws, ws_bytes, stream);
-  if (st != FP4_OK) return st;
-  st = fp4_gemm(&sv->dyq, &sv->wq_t, 1.0f, dx, K, cfg->out_dtype, nullptr, ws, ws_bytes, stream);
-  if (st != FP4_OK) return st;
-  return fp4_gemm(&sv->dyq_t, &sv->xq_t, 1.0f, dw, K, FP4_OUT_F32, nullptr, ws, ws_bytes, stream);
+  for (const bool dry : {true, false}) {
+    st = quantize_impl(dy, M, N, N, &pd, &sv->dyq, &sv->dyq_t, ws, ws_bytes, stream, dry);
+    if (st != FP4_OK) return st;
+    st = gemm_impl(&sv->dyq, &sv->wq_t, 1.0f, dx, K, cfg->out_dtype, nullptr, ws, ws_bytes,
+                   stream, dry);
+    if (st != FP4_OK) return st;
+    st = gemm_impl(&sv->dyq_t, &sv->xq_t, 1.0f, dw, K, FP4_OUT_F32, nullptr, ws, ws_bytes,
+                   stream, dry);
+    if (st != FP4_OK) return st;
+  }
+  return FP4_OK;
 }
 
 fp4_status fp4_read_device_status(const void* ws, void* stream) {

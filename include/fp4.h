@@ -227,13 +227,18 @@ typedef struct fqt_saved {
 } fqt_saved;
 
 /* Forward: quantize X (row-wise and transposed) and W (both orientations),
- * then Y = fprop.  x, w BF16; y of cfg->out_dtype, [M, N] dense. */
+ * then Y = fprop.  x, w BF16; y of cfg->out_dtype, [M, N] dense.  The
+ * shape, alignment and workspace rules are those of the fp4_quantize and
+ * fp4_gemm calls it makes (M, N multiples of 128, K of 128 for the backward's
+ * outputs); all of them are checked before the first is enqueued, so an
+ * argument error leaves the stream untouched. */
 fp4_status fqt_linear_fwd(const fqt_linear_cfg* cfg, int64_t M, int64_t N, int64_t K,
                           const void* x, const void* w, void* y, fqt_saved* saved,
                           void* ws, size_t ws_bytes, void* stream);
 
 /* Backward: quantize dY (row-wise and transposed), then dX = dgrad
- * ([M, K], cfg->out_dtype) and dW = wgrad ([N, K], FP32). */
+ * ([M, K], cfg->out_dtype) and dW = wgrad ([N, K], FP32), from the operands
+ * fqt_linear_fwd left in `saved`.  Argument errors as for the forward. */
 fp4_status fqt_linear_bwd(const fqt_linear_cfg* cfg, int64_t M, int64_t N, int64_t K,
                           const void* dy, fqt_saved* saved, void* dx, float* dw,
                           void* ws, size_t ws_bytes, void* stream);
@@ -299,9 +304,9 @@ int32_t fp4_abi_version(void);
  * MMA thread, the three scale-factor copies into tensor memory that one MMA
  * of a GEMM K step needs; variants 4 and 5 issue the same copies from a
  * second warp concurrently with the MMAs.  Writes the
- * achieved TFLOP/s.  The measured rate is the denominator the GEMM's
- * tensor-pipe fraction is reported against ("FP4" page, Hardware: FP4 on
- * fifth-generation Tensor Cores). */
+ * achieved TFLOP/s: what the tensor pipe sustains with and without the
+ * scale-factor traffic, the context for the GEMM's rate ("FP4" page,
+ * Hardware: FP4 on fifth-generation Tensor Cores). */
 fp4_status fp4_mma_rate(int32_t variant, int32_t iters, float* tflops_out, void* ws,
                         size_t ws_bytes, void* stream);
 

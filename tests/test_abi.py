@@ -128,3 +128,23 @@ def test_gemm_quant_and_noise_argument_errors(lib):
     assert lib.fp4_quant_noise(x, 32, 64, 64, C.byref(q), C.c_void_p((1 << 24) + 4), None, 0,
                                None) == 3
     assert lib.fp4_quant_noise(x, 32, 64, 64, C.byref(_q(32, 64, 5)), sums, None, 0, None) == 4
+
+
+def test_linear_layer_rejects_before_any_launch(lib):
+    """fqt_linear_fwd / fqt_linear_bwd check every one of their quantize and
+    GEMM calls before enqueuing the first: a shape only the GEMM rejects
+    (M = 96, not a multiple of 128) returns FP4_ERR_SHAPE, not the CUDA error
+    the X quantizer's first enqueue would meet on a machine without a GPU, and
+    the library's launch counter does not move."""
+    M, N, K = 96, 128, 128
+    sv = F.SavedC(_q(M, K), _q(K, M), _q(N, K, 0, 1), _q(K, N, 0, 1), _q(M, N), _q(N, M))
+    cfg = F.linear_cfg(F.NVFP4)
+    x = C.c_void_p(1 << 20)
+    ws = C.c_void_p(1 << 21)
+    n0 = lib.fp4_kernel_launches()
+    assert lib.fqt_linear_fwd(C.byref(cfg), M, N, K, x, x, x, C.byref(sv), ws, 256, None) == 2
+    assert lib.fqt_linear_bwd(C.byref(cfg), M, N, K, x, C.byref(sv), x, x, ws, 256, None) == 2
+    # a missing workspace is only a GEMM error too
+    sv2 = F.SavedC(_q(128, K), _q(K, 128), _q(N, K, 0, 1), _q(K, N, 0, 1), _q(128, N), _q(N, 128))
+    assert lib.fqt_linear_fwd(C.byref(cfg), 128, N, K, x, x, x, C.byref(sv2), None, 0, None) == 5
+    assert lib.fp4_kernel_launches() == n0
