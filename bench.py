@@ -146,6 +146,19 @@ class Layer:
         self.dw = torch.empty((N, K), dtype=torch.float32, device=device)
 
 
+def step_config(fmt: str, wgrad_rht: bool, world: int, dp_allreduce: bool) -> dict:
+    """The `config` of the step's JSON line, shared by both arms."""
+    nv = fmt == "nvfp4"
+    rht = ("wgrad 16-pt" if wgrad_rht else "off") if nv else "all GEMMs 32-pt"
+    return {"workload": "Llama-7B linear layers fwd+bwd (QKVO x4 4096x4096, gate/up x2 "
+                        "11008x4096, down 11008->4096), tokens 32768 (bs 64 x seq 512)",
+            "format": fmt, "rounding": "RTN fwd, SR bwd/update" if nv else "RTN fwd/bwd",
+            "weights": "16x16 tiles" if nv else "1x32", "rht": rht,
+            "l2": "inputs larger than L2 (no flush)",
+            "parallelism": f"dp x{world}, dW all-reduce (NCCL, overlapped)" if dp_allreduce
+            else f"replicas x{world}"}
+
+
 def make_layers(F, cfg, device, seed):
     import fqt_synth as S
     cache = {}
@@ -307,12 +320,16 @@ def e2e_run(F, layers, cache, cfg, ws, steps, device, dp=None):
     return ms, h2d, d2h
 
 
-def cpu_baseline(rows_sample: int = 1024, cols_sample: int = 2048, seed: int = 0, cache=None):
+def cpu_baseline(rows_sample: int = 1024, cols_sample: int = 2048, seed: int = 0, cache=None,
+                 fmt: str = "nvfp4", wgrad_rht: bool = False):
     """The oracle, as it stands, on a bounded sample of the same workload: for
     each of the 7 layers the first `rows_sample` tokens and the first
-    `cols_sample` output features (X[:r], W[:c], dY[:r, :c]): NVFP4 quantize
-    of X, W, dY in both orientations, then the three GEMMs in float64.
-    Throughput in the metric's unit: 6 * r * c * K flops per second."""
+    `cols_sample` output features (X[:r], W[:c], dY[:r, :c]): the step's
+    quantizations of X, W, dY in both orientations (NVFP4: RTN X and 16x16
+    W, SR dY and X^T, optionally the 16-point rotation on the wgrad operands;
+    MXFP4: RTN with the 32-point rotation everywhere), then the three GEMMs
+    in float64.  Throughput in the metric's unit: 6 * r * c * K flops per
+    second."""
     import fqt_synth as S
     import oracle as O
     t_total = 0.0
@@ -321,6 +338,8 @@ def cpu_baseline(rows_sample: int = 1024, cols_sample: int = 2048, seed: int = 0
     if cache is None:
         cache = {}
     r, c = rows_sample, cols_sample
+    nv = fmt == "nvfp4"
+    rw = 16 if wgrad_rht else 0
     for name, N, K in LAYERS:
         if (N, K) not in seen:
             if (N, K) not in cache:
@@ -330,22 +349,32 @@ def cpu_baseline(rows_sample: int = 1024, cols_sample: int = 2048, seed: int = 0
         X, W, dY = seen[(N, K)]
         T = lambda a: np.ascontiguousarray(a.T)
         t0 = time.perf_counter()
-        qx = O.nvfp4_quantize_1d(X)
-        qxt = O.nvfp4_quantize_1d(T(X), "sr", sr_seed=seed, sr_stream=3)
-        qw = O.nvfp4_quantize_2d(W)
-        qwt = O.nvfp4_quantize_2d(T(W))
-        qd = O.nvfp4_quantize_1d(dY, "sr", sr_seed=seed, sr_stream=1)
-        qdt = O.nvfp4_quantize_1d(T(dY), "sr", sr_seed=seed, sr_stream=2)
-        deq = lambda q, b=(1, 16): O.dequantize(q["codes"], q["scales"], b)
-        O.gemm(deq(qx), deq(qw, (16, 16)), s_dec_a=qx["s_dec"], s_dec_b=qw["s_dec"])
-        O.gemm(deq(qd), deq(qwt, (16, 16)), s_dec_a=qd["s_dec"], s_dec_b=qwt["s_dec"])
+        if nv:
+            qx = O.nvfp4_quantize_1d(X)
+            qxt = O.nvfp4_quantize_1d(T(X), "sr", rht_n=rw, rht_seed=seed, sr_seed=seed,
+                                      sr_stream=3)
+            qw = O.nvfp4_quantize_2d(W)
+            qwt = O.nvfp4_quantize_2d(T(W))
+            qd = O.nvfp4_quantize_1d(dY, "sr", sr_seed=seed, sr_stream=1)
+            qdt = O.nvfp4_quantize_1d(T(dY), "sr", rht_n=rw, rht_seed=seed, sr_seed=seed,
+                                      sr_stream=2)
+            deq = lambda q, b=(1, 16): O.dequantize(q["codes"], q["scales"], b)
+            wb = (16, 16)
+        else:
+            mx = lambda a: O.mxfp4_quantize(a, "rtn", rht_n=32, rht_seed=seed)
+            qx, qxt, qw, qwt, qd, qdt = mx(X), mx(T(X)), mx(W), mx(T(W)), mx(dY), mx(T(dY))
+            deq = lambda q, b=None: O.dequantize(q["codes"], q["scales"], (1, 32), True)
+            wb = None
+        O.gemm(deq(qx), deq(qw, wb), s_dec_a=qx["s_dec"], s_dec_b=qw["s_dec"])
+        O.gemm(deq(qd), deq(qwt, wb), s_dec_a=qd["s_dec"], s_dec_b=qwt["s_dec"])
         O.gemm(deq(qdt), deq(qxt), s_dec_a=qdt["s_dec"], s_dec_b=qxt["s_dec"])
         t_total += time.perf_counter() - t0
         flops += 6 * r * c * K
     return {"value": flops / t_total / 1e12, "unit": "TFLOP/s", "cores": O.num_threads(),
             "kind": "oracle", "seconds": round(t_total, 2),
             "sample": f"first {r} of {M_TOKENS} tokens x first {c} output features of each of "
-                      "the 7 layers: NVFP4 quantize (both orientations) + 3 float64 GEMMs"}
+                      f"the 7 layers: {fmt.upper()} quantize (both orientations) + 3 float64 "
+                      "GEMMs"}
 
 
 def run_ours(args, rank, world, device):
@@ -439,14 +468,8 @@ def run_ours(args, rank, world, device):
                  "fp4(e2m1)+e8m0 scales, fp32 accumulate",
         "data": "synthetic (seeded): X N(0,1) with 1% Student-t(3) channels, W N(0,0.02^2), "
                 "dY N(0,1e-6)",
-        "config": {"workload": "Llama-7B linear layers fwd+bwd (QKVO x4 4096x4096, gate/up x2 "
-                               "11008x4096, down 11008->4096), tokens 32768 (bs 64 x seq 512)",
-                   "format": args.fmt, "rounding": "RTN fwd, SR bwd/update" if fmt == F.NVFP4
-                   else "RTN fwd/bwd", "weights": "16x16 tiles" if fmt == F.NVFP4 else "1x32",
-                   "rht": {0: "off", 4: "wgrad 16-pt", 7: "all GEMMs 32-pt"}.get(cfg.rht_mask),
-                   "l2": "inputs larger than L2 (no flush)",
-                   "parallelism": f"dp x{world}, dW all-reduce (NCCL, overlapped)"
-                   if dp is not None else f"replicas x{world}"},
+        "config": step_config(args.fmt, bool(args.wgrad_rht and fmt == F.NVFP4), world,
+                              dp is not None),
         "roofline": {"kernel": "fp4_gemm_sfst_kernel (tcgen05 block-scaled, scales staged by tcgen05.st)", "bound": "tensor",
                      "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1),
                      "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4),
@@ -479,9 +502,9 @@ def run_reference(args):
     steps = []
     cache = {}                    # the synthetic layers are generated once, not per step
     for _ in range(args.warmup):
-        cpu_baseline(rows, cols, args.seed, cache)
+        cpu_baseline(rows, cols, args.seed, cache, args.fmt, args.wgrad_rht)
     for _ in range(args.steps):
-        steps.append(cpu_baseline(rows, cols, args.seed, cache))
+        steps.append(cpu_baseline(rows, cols, args.seed, cache, args.fmt, args.wgrad_rht))
     v = statistics.median(s["value"] for s in steps)
     secs = sum(s["seconds"] for s in steps)
     flops_step = sum(6 * M_TOKENS * N * K for _, N, K in LAYERS)
@@ -492,9 +515,8 @@ def run_reference(args):
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms, 1), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic (seeded)",
-            "config": {"workload": "Llama-7B linear layers fwd+bwd, tokens 32768; each step a "
-                                   f"bounded sample of {rows} tokens x {cols} "
-                                   "output features per layer"},
+            "config": step_config(args.fmt, bool(args.wgrad_rht and args.fmt == "nvfp4"), 1,
+                                  args.dp_allreduce),
             "cpu_baseline": cb, "seconds_total": round(secs, 1),
             "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -830,7 +852,8 @@ def main():
     torch.cuda.set_device(device)
     out, cache = run_ours(args, rank, world, device)
     if rank == 0 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(args.ref_rows or 1024, args.ref_cols or 2048, args.seed, cache)
+        out["cpu_baseline"] = cpu_baseline(args.ref_rows or 1024, args.ref_cols or 2048, args.seed,
+                                           cache, args.fmt, args.wgrad_rht)
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
