@@ -261,7 +261,9 @@ def e2e_run(F, layers, cache, cfg, ws, steps, device, dp=None):
     and device-to-host copies of layer i - 1 run while layer i computes, and
     the two copy directions overlap each other.  Events order each layer's
     buffers: its inputs are overwritten only after the previous step's
-    compute read them, its outputs only after the previous step's copy-out."""
+    compute read them, its outputs only after the previous step's copy-out.
+    Returns (ms per step, H2D bytes, D2H bytes, the pinned host buffers by
+    layer shape)."""
     host = {}
     for (N, K), src in cache.items():
         host[(N, K)] = {
@@ -317,7 +319,7 @@ def e2e_run(F, layers, cache, cfg, ws, steps, device, dp=None):
     b.record(d2h_s)
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / steps
-    return ms, h2d, d2h
+    return ms, h2d, d2h, host
 
 
 def cpu_baseline(rows_sample: int = 1024, cols_sample: int = 2048, seed: int = 0, cache=None,
@@ -449,7 +451,7 @@ def run_ours(args, rank, world, device):
 
     e2e = None
     if not args.no_e2e:
-        e_ms, h2d, d2h = e2e_run(F, layers, cache, cfg, ws, args.e2e_steps, device, dp)
+        e_ms, h2d, d2h, _host = e2e_run(F, layers, cache, cfg, ws, args.e2e_steps, device, dp)
         e_max = max_over_ranks(e_ms, device, world)
         e2e = {"value": round(whole_job_rate(flops_step, world, e_max) / 1e12, 2),
                "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
