@@ -6,20 +6,22 @@
  *
  * What is computed (page title, section):
  *   - "FP4" (Robots Atlas), How it works: values are cast to 4-bit E2M1;
- *     a tensor is split into small blocks (16 values for NVFP4, 32 for
- *     MXFP4), each with its own scale (E4M3 for NVFP4, E8M0 for MXFP4);
+ *     runs of 16 (NVFP4) or 32 (MXFP4) consecutive values share one scale
+ *     each (E4M3 for NVFP4, E8M0 for MXFP4);
  *     NVFP4 adds one FP32 scale for the whole tensor; matrix products run
  *     on the tensor cores in FP4 and accumulate in higher precision; random
  *     Hadamard transforms, two-dimensional quantization and stochastic
  *     rounding of gradients stabilise training.
- *   - "FP4" (Robots Atlas), Components: the E2M1 levels 0, 0.5, 1, 1.5, 2,
- *     3, 4, 6 and their negatives; NVFP4 and MXFP4 block formats.
+ *   - "FP4" (Robots Atlas), Components: the eight E2M1 magnitudes 0, 0.5,
+ *     1, 1.5, 2, 3, 4, 6, each with either sign; NVFP4 and MXFP4 block
+ *     formats.
  *   - "FP4 All the Way: Fully Quantized Training of LLMs", Key points:
  *     NVFP4, round-to-nearest in the forward pass, stochastic rounding in
  *     the backward and update passes.
  *   - "Quartet: Native FP4 Training Can Be Optimal for Large Language
- *     Models", Approach: all three linear-layer GEMMs in FP4, round-to-
- *     nearest backward with block-wise Hadamard rotations (the MXFP4 mode).
+ *     Models", Approach: fprop, dgrad and wgrad each computed from FP4
+ *     operands, round-to-nearest backward with block-wise Hadamard
+ *     rotations (the MXFP4 mode).
  *
  * Conventions shared by every entry point:
  *   - Every tensor pointer is DEVICE memory owned by the caller.  The

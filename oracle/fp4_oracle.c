@@ -83,9 +83,9 @@ static void parallel_rows(row_fn fn, void* ctx, int64_t nrows) {
 }
 
 /* ------------------------------------------------------------------------ */
-/* E2M1: 1 sign bit, 2 exponent bits, 1 mantissa bit.                       */
-/* [FP4] Components, "E2M1 format": levels 0, 0.5, 1, 1.5, 2, 3, 4, 6 and   */
-/* their negatives; range about -6..+6.                                     */
+/* E2M1: sign in bit 3, a two-bit exponent in bits 2-1, mantissa in bit 0.  */
+/* [FP4] Components, "E2M1 format": eight magnitudes 0, 0.5, 1, 1.5, 2, 3, */
+/* 4, 6, each with either sign, so the format spans +-6.                    */
 /* ------------------------------------------------------------------------ */
 double orc_e2m1_value(uint8_t code) {
   int s = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
@@ -175,7 +175,8 @@ uint8_t orc_e4m3_rne_sat(float t) {
 
 /* ------------------------------------------------------------------------ */
 /* E8M0: unsigned power-of-two scale 2^(b-127); 0xFF is NaN.                */
-/* [FP4] Components, "MXFP4": shared E8M0 scale, power of two only.         */
+/* [FP4] Components, "MXFP4": one E8M0 scale per 32-value block, which can  */
+/* only be a power of two.                                                  */
 /* ------------------------------------------------------------------------ */
 double orc_e8m0_value(uint8_t b) {
   if (b == 0xFF) return NAN;
