@@ -148,3 +148,20 @@ def test_linear_layer_rejects_before_any_launch(lib):
     sv2 = F.SavedC(_q(128, K), _q(K, 128), _q(N, K, 0, 1), _q(K, N, 0, 1), _q(128, N), _q(N, 128))
     assert lib.fqt_linear_fwd(C.byref(cfg), 128, N, K, x, x, x, C.byref(sv2), None, 0, None) == 5
     assert lib.fp4_kernel_launches() == n0
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """Without the built library every entry point raises: there is no CPU
+    fallback behind the binding."""
+    import torch
+    monkeypatch.setattr(F, "LIB_PATH", str(tmp_path / "libfp4fqt.so"))
+    monkeypatch.setattr(F, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        F.load()
+    with pytest.raises(RuntimeError, match="missing"):
+        F.qtensor_sizes(16, 16)
+    with pytest.raises(RuntimeError, match="missing"):
+        F.linear_cfg(F.NVFP4)
+    x = torch.zeros((16, 16), dtype=torch.bfloat16)
+    with pytest.raises((RuntimeError, AssertionError)):
+        F.fp4_quantize(x, None)
