@@ -16,13 +16,22 @@ FLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-pthread", "-ffp-contract=off",
          "-fno-fast-math", "-fexcess-precision=standard", "-Wall", "-Wextra"]
 
 
+def compile_to(src: str, out: str) -> str:
+    """Compile an oracle source file with the oracle's flags."""
+    subprocess.run(["gcc", *FLAGS, "-o", out, src, "-lm"], check=True)
+    return out
+
+
 def build(force: bool = False) -> str:
+    # The mutation test points this at a deliberately broken copy of the
+    # oracle, compiled by compile_to, to check that the pins catch it.
+    override = os.environ.get("FP4_ORACLE_LIB")
+    if override:
+        return override
     if (not force and os.path.exists(LIB)
             and os.path.getmtime(LIB) >= os.path.getmtime(SRC)):
         return LIB
-    cmd = ["gcc", *FLAGS, "-o", LIB, SRC, "-lm"]
-    subprocess.run(cmd, check=True)
-    return LIB
+    return compile_to(SRC, LIB)
 
 
 if __name__ == "__main__":

@@ -135,6 +135,49 @@ def test_nvfp4_row_offset_and_sr_index():
                           O.nvfp4_quantize_1d(lat)["codes"])
 
 
+def _unit_scale_blocks(rng, R, C, bs):
+    """x[R, C] whose every bs-block has max |x| = 6 exactly and whose other
+    values are arbitrary binary32 numbers in (-6, 6): with a tensor amax of
+    2688 (NVFP4: s_enc = 1, block scale E4M3(1) = 1) or directly (MXFP4:
+    scale 2^(floor(log2 6) - 2) = 1) every value reaches E2M1 rounding
+    unscaled."""
+    x = rng.uniform(-6.0, 6.0, (R, C)).astype(np.float32)
+    x[:, ::bs] = np.where(rng.random((R, C // bs)) < 0.5, -6.0, 6.0)
+    return x
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
+def test_sr_draw_index_is_row_major_in_the_operand(fmt):
+    """Element (r, c) of rows starting at row_offset of an [*, C] operand is
+    rounded with draw (row_offset + r) * C + c of its stream (the layout
+    reading), checked value by value where the scales are exactly 1."""
+    rng = np.random.default_rng(31)
+    R, C, off, seed, stream = 3, 64, 5, 11, 2
+    bs = 16 if fmt == "nvfp4" else 32
+    x = _unit_scale_blocks(rng, R, C, bs)
+    if fmt == "nvfp4":
+        q = O.nvfp4_quantize_1d(x, "sr", sr_seed=seed, sr_stream=stream, amax_in=2688.0,
+                                row_offset=off)
+        assert np.all(q["scales"] == O.e4m3_rne_sat(np.float32(1.0))[0])
+    else:
+        q = O.mxfp4_quantize(x, "sr", sr_seed=seed, sr_stream=stream, row_offset=off)
+        assert np.all(q["scales"] == 127)
+    u = O.draws(seed, stream, off * C, R * C).reshape(R, C)
+    want = O.e2m1_sr(x.reshape(-1), u.reshape(-1)).reshape(R, C)
+    assert np.array_equal(_codes(q["codes"]), want)
+
+
+def test_amax_is_of_magnitudes():
+    """The tensor amax is max |x|: a tensor whose extreme is negative."""
+    x = np.array([[-5.0, 1.0, 2.0, -0.5] * 4], np.float32)
+    assert O.amax(x) == 5.0
+    assert O.nvfp4_quantize_1d(x)["amax"] == 5.0
+    assert O.nvfp4_quantize_2d(np.tile(x, (16, 1)))["amax"] == 5.0
+    y = np.random.default_rng(32).standard_normal((8, 32)).astype(np.float32)
+    y[3, 9] = -40.0
+    assert O.amax(y) == 40.0
+
+
 def test_nvfp4_rht_amax_is_of_rotated_tensor():
     rng = np.random.default_rng(14)
     x = rng.standard_normal((4, 64)).astype(np.float32)

@@ -48,6 +48,28 @@ def test_up_probability_is_exact_fraction_of_gap():
                                np.array([0, 0, 1], np.uint32)))) == [6.0, 0.5, 0.0]
 
 
+def test_extreme_draws_decide_every_interior_value():
+    """Strictly between two levels 0 < p < 1, so ceil(p * 2^32) lies in
+    [1, 2^32 - 1]: the draw 0 always rounds up and the draw 2^32 - 1 never
+    does, down to p of a single binary32 subnormal (a rounded-down threshold
+    would send the smallest p to the lower level with every draw)."""
+    rng = np.random.default_rng(7)
+    v = np.concatenate([rng.uniform(-6.0, 6.0, 4096),
+                        2.0 ** -np.arange(2, 150, dtype=np.float64),
+                        -(2.0 ** -np.arange(2, 150, dtype=np.float64)),
+                        rng.uniform(0.0, 1e-30, 256)]).astype(np.float32)
+    lv = np.array(LEVELS)
+    keep = (np.abs(v) > 0) & (np.abs(v) < 6.0) & ~np.isin(np.abs(v).astype(np.float64), lv)
+    v = v[keep]
+    a = np.abs(v).astype(np.float64)
+    hi = np.array([lv[lv > x].min() for x in a])
+    lo = np.array([lv[lv < x].max() for x in a])
+    up = np.abs(_val(O.e2m1_sr(v, np.zeros(v.size, np.uint32))))
+    down = np.abs(_val(O.e2m1_sr(v, np.full(v.size, 2**32 - 1, np.uint32))))
+    assert np.array_equal(up, hi)
+    assert np.array_equal(down, lo)
+
+
 def test_monotone_in_v_for_fixed_draw():
     rng = np.random.default_rng(4)
     v = np.sort(rng.uniform(-7, 7, 5000).astype(np.float32))
