@@ -80,6 +80,21 @@ MUTANTS = [
      "float v = fabsf(q->x[(i * 16 + a) * C + j * 16 + b]);",
      "float v = fabsf(q->x[(i * 16) * C + j * 16 + b]);", 0),
     ("floor(log2) of subnormals", "return k - 149;", "return k - 150;", 0),
+    ("floor(log2) of normals", "if (E > 0) return E - 127;", "if (E > 0) return E - 126;", 0),
+    ("E4M3 subnormal exponent", "ldexp((double)m / 8.0, -6)", "ldexp((double)m / 8.0, -7)", 0),
+    ("E2M1 RTN clamps at 5", "if (a > 8.0) a = 8.0;", "if (a > 5.0) a = 5.0;", 0),
+    ("2-D block scale divides by 4, not 6", "float t = (bmax * q->s_enc) / 6.0f;",
+     "float t = (bmax * q->s_enc) / 4.0f;", 1),
+    ("2-D block reciprocal inverted", "float inv = (sf == 0) ? 0.0f : q->s_enc / sfv;",
+     "float inv = (sf == 0) ? 0.0f : sfv / q->s_enc;", 1),
+    ("dequantize with the other scale format",
+     "double sv = is_e8m0 ? orc_e8m0_value(s) : orc_e4m3_value(s);",
+     "double sv = is_e8m0 ? orc_e4m3_value(s) : orc_e8m0_value(s);", 0),
+    ("MXFP4 exponent clamp at -126", "if (e < -127) e = -127;", "if (e < -126) e = -126;", 0),
+    ("zero tensor decodes with scale 0", "if (A == 0.0f) { *s_enc = 1.0f; *s_dec = 1.0f; return; }",
+     "if (A == 0.0f) { *s_enc = 1.0f; *s_dec = 0.0f; return; }", 0),
+    ("reciprocal of a zero scale not zero", "float inv = (sf == 0) ? 0.0f : q->s_enc / sfv;",
+     "float inv = (sf == 0) ? 1.0f : q->s_enc / sfv;", 0),
 ]
 
 

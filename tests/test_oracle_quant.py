@@ -114,6 +114,14 @@ def test_nvfp4_special_cases():
     # a supplied amax is used as given
     q2 = O.nvfp4_quantize_1d(x, amax_in=80.0)
     assert q2["amax"] == np.float32(80.0) and q2["scales"][5, 1] < 0x7E
+    # a block whose scale underflows E4M3 (b * s_enc / 6 below 2^-10) has
+    # scale code 0 and encodes to zeros, keeping only the signs
+    y = np.zeros((1, 32), np.float32)
+    y[0, 0] = 1.0e6                       # s_enc = 2688 / 1e6
+    y[0, 16:] = np.linspace(-1.0, 1.0, 16, dtype=np.float32)
+    q3 = O.nvfp4_quantize_1d(y)
+    assert q3["scales"][0, 1] == 0
+    assert np.all(_codes(q3["codes"])[0, 16:] & 7 == 0)
 
 
 def test_nvfp4_row_offset_and_sr_index():
@@ -203,9 +211,15 @@ def test_nvfp4_2d_tile_scale_and_transpose():
     # one scale per 16x16 tile: the tile scale equals a 1-D quantization of
     # the flattened tile with the same tensor amax
     s_enc, _ = O.nvfp4_global_scales(q["amax"])
-    tile = w[16:32, 32:48]
-    t = np.float32(np.float32(np.abs(tile).max() * s_enc) / np.float32(6.0))
-    assert q["scales"][1, 2] == O.e4m3_rne_sat([t])[0]
+    codes = _codes(q["codes"])
+    for i in range(3):
+        for j in range(4):
+            tile = w[16 * i:16 * i + 16, 16 * j:16 * j + 16]
+            t = np.float32(np.float32(np.abs(tile).max() * s_enc) / np.float32(6.0))
+            assert q["scales"][i, j] == O.e4m3_rne_sat([t])[0], (i, j)
+            # the tile's largest magnitude lands on the top level, 6
+            a, b = np.unravel_index(np.argmax(np.abs(tile)), tile.shape)
+            assert abs(O.e2m1_value(int(codes[16 * i + a, 16 * j + b]))) == 6.0, (i, j)
 
 
 def test_mxfp4_scale_rule_and_bounds():
