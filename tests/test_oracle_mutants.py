@@ -153,3 +153,43 @@ def test_gemm_reference_mutants_are_caught(monkeypatch):
             Q.test_gemm_reference_exact_on_small_case()
     monkeypatch.setattr(O, "gemm", orig)
     Q.test_gemm_reference_exact_on_small_case()
+
+
+def _fails(fn) -> bool:
+    try:
+        fn()
+    except AssertionError:
+        return True
+    return False
+
+
+def test_quant_noise_mutants_are_caught(monkeypatch):
+    """The noise diagnostic's reference without the tensor decode scale, with
+    |error| summed instead of its square, or with the dequantized signal in
+    place of the input's, fails one of its pins."""
+    import numpy as np
+    import test_oracle_quant as Q
+    orig = O.quant_noise
+    pins = (Q.test_quant_noise_closed_form_mxfp4_block,
+            Q.test_quant_noise_zero_for_representable_blocks,
+            Q.test_quant_noise_matches_independent_decode_nvfp4)
+
+    def no_sdec(x, codes, scales, s_dec, block=(1, 16), e8m0=False):
+        return orig(x, codes, scales, 1.0, block, e8m0)
+
+    def abs_error(x, codes, scales, s_dec, block=(1, 16), e8m0=False):
+        x = np.asarray(x, dtype=np.float64)
+        d = O.dequantize(codes, scales, block, e8m0) * float(s_dec) - x
+        return float(np.sum(x * x)), float(np.sum(np.abs(d)))
+
+    def signal_of_deq(x, codes, scales, s_dec, block=(1, 16), e8m0=False):
+        deq = O.dequantize(codes, scales, block, e8m0) * float(s_dec)
+        d = deq - np.asarray(x, dtype=np.float64)
+        return float(np.sum(deq * deq)), float(np.sum(d * d))
+
+    for mutant in (no_sdec, abs_error, signal_of_deq):
+        monkeypatch.setattr(O, "quant_noise", mutant)
+        assert any(_fails(p) for p in pins), mutant.__name__
+    monkeypatch.setattr(O, "quant_noise", orig)
+    for p in pins:
+        p()
