@@ -9,6 +9,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <climits>
 #include <cstdint>
 #include <cstring>
 
@@ -275,6 +276,11 @@ fp4_status fp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
   return quantize_impl(x, rows, cols, ld, p, out, out_t, ws, ws_bytes, stream, false);
 }
 
+// The GEMM kernel numbers its 128 x 256 output tiles with 32-bit integers.
+static bool gemm_tiles_fit(int64_t M, int64_t N) {
+  return (M / 128) * ((N + 255) / 256) <= (int64_t)INT32_MAX;
+}
+
 // fp4_gemm; with `dry` it only validates the arguments.
 static fp4_status gemm_impl(const fp4_qtensor* a, const fp4_qtensor* b, float alpha, void* c,
                             int64_t ldc, int32_t out_dtype, float* c_amax, void* ws,
@@ -289,6 +295,7 @@ static fp4_status gemm_impl(const fp4_qtensor* a, const fp4_qtensor* b, float al
   if (b->cols != K) return FP4_ERR_SHAPE;
   if (M <= 0 || N <= 0 || K <= 0 || M % 128 || N % 128 || K % 64) return FP4_ERR_SHAPE;
   if (M > (1ll << 30) || N > (1ll << 30) || K > (1ll << 30)) return FP4_ERR_SHAPE;
+  if (!gemm_tiles_fit(M, N)) return FP4_ERR_SHAPE;
   const int64_t esize = out_dtype == FP4_OUT_F32 ? 4 : 2;
   if (ldc < N || (ldc * esize) % 16 || !aligned16(c)) return FP4_ERR_ALIGN;
   if (!aligned16(a->codes) || !aligned16(b->codes) || !aligned16(a->scales_mma) ||
@@ -310,6 +317,7 @@ fp4_status fp4_gemm(const fp4_qtensor* a, const fp4_qtensor* b, float alpha, voi
   return gemm_impl(a, b, alpha, c, ldc, out_dtype, c_amax, ws, ws_bytes, stream, false);
 }
 
+
 fp4_status fp4_gemm_quant(const fp4_qtensor* a, const fp4_qtensor* b, float alpha,
                           const float* out_amax_in, fp4_qtensor* out, float* c_amax, void* ws,
                           size_t ws_bytes, void* stream) {
@@ -326,6 +334,7 @@ fp4_status fp4_gemm_quant(const fp4_qtensor* a, const fp4_qtensor* b, float alph
   if (b->cols != K || out->rows != M || out->cols != N) return FP4_ERR_SHAPE;
   if (M <= 0 || N <= 0 || K <= 0 || M % 128 || N % 128 || K % 64) return FP4_ERR_SHAPE;
   if (M > (1ll << 30) || N > (1ll << 30) || K > (1ll << 30)) return FP4_ERR_SHAPE;
+  if (!gemm_tiles_fit(M, N)) return FP4_ERR_SHAPE;
   if (!aligned16(a->codes) || !aligned16(b->codes) || !aligned16(a->scales_mma) ||
       !aligned16(b->scales_mma) || !aligned16(out->codes) ||
       (reinterpret_cast<uintptr_t>(out->scales_mma) & 3u) ||
@@ -464,3 +473,11 @@ fp4_status fp4_clear_device_status(void* ws, void* stream) {
 }
 
 }  // extern "C"
+
+namespace fp4impl {
+fp4_status gemm_validate(const fp4_qtensor* a, const fp4_qtensor* b, const void* c, int64_t ldc,
+                         int32_t out_dtype, const void* ws, size_t ws_bytes) {
+  return gemm_impl(a, b, 1.0f, const_cast<void*>(c), ldc, out_dtype, nullptr,
+                   const_cast<void*>(ws), ws_bytes, nullptr, true);
+}
+}  // namespace fp4impl

@@ -94,6 +94,9 @@ struct GemmArgs {
   uint32_t* status;
 };
 fp4_status gemm_launch(const GemmArgs& g, cudaStream_t s);
+// Every argument check of fp4_gemm, with nothing enqueued (api.cu).
+fp4_status gemm_validate(const fp4_qtensor* a, const fp4_qtensor* b, const void* c, int64_t ldc,
+                         int32_t out_dtype, const void* ws, size_t ws_bytes);
 // Scale factors staged into TMEM by tcgen05.st warps (gemm_sfst.cu).
 fp4_status gemm_launch_sfst(const GemmArgs& g, cudaStream_t s);
 

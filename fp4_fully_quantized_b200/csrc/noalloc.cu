@@ -61,6 +61,9 @@ extern "C" fp4_status fp4_gemm_noalloc(const fp4_qtensor* a, const fp4_qtensor* 
   void* scratch = nullptr;
   fp4_status st = scratch_for_current_device(&scratch);
   if (st != FP4_OK) return st;
+  // Every argument error returns before the clear below is enqueued.
+  st = fp4impl::gemm_validate(a, b, c, ldc, out_dtype, scratch, kNoAllocScratchBytes);
+  if (st != FP4_OK) return st;
   // The array keeps the previous call's contents: the status block must start
   // at zero for this call's device conditions to be recorded.
   if (cudaMemsetAsync(scratch, 0, sizeof(fp4impl::DeviceStatus),

@@ -165,3 +165,17 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     x = torch.zeros((16, 16), dtype=torch.bfloat16)
     with pytest.raises((RuntimeError, AssertionError)):
         F.fp4_quantize(x, None)
+
+
+def test_gemm_rejects_tile_counts_beyond_32_bits(lib):
+    """Shapes within the per-dimension limits whose 128 x 256 tile count does
+    not fit the kernel's 32-bit tile numbering are rejected on the host."""
+    big = 1 << 30
+    a, b = _q(big, 128), _q(big, 128)
+    c = C.c_void_p(1 << 22)
+    ws = C.c_void_p(1 << 21)
+    assert lib.fp4_gemm(C.byref(a), C.byref(b), 1.0, c, big, 0, None, ws, 256, None) == 2
+    out = _q(big, big)
+    amax = C.c_void_p(1 << 23)
+    assert lib.fp4_gemm_quant(C.byref(a), C.byref(b), 1.0, amax, C.byref(out), None, ws, 256,
+                              None) == 2
