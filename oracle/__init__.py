@@ -38,6 +38,7 @@ def lib():
         u8p = np.ctypeslib.ndpointer(np.uint8, flags="C_CONTIGUOUS")
         u32p = np.ctypeslib.ndpointer(np.uint32, flags="C_CONTIGUOUS")
         f64p = np.ctypeslib.ndpointer(np.float64, flags="C_CONTIGUOUS")
+        u16p = np.ctypeslib.ndpointer(np.uint16, flags="C_CONTIGUOUS")
         i64, u64, u32, i32 = C.c_int64, C.c_uint64, C.c_uint32, C.c_int
         L.orc_e2m1_value.restype = C.c_double
         L.orc_e2m1_value.argtypes = [C.c_uint8]
@@ -48,7 +49,7 @@ def lib():
         L.orc_e2m1_rtn.restype = C.c_uint8
         L.orc_e2m1_rtn.argtypes = [C.c_float]
         L.orc_e2m1_sr.restype = C.c_uint8
-        L.orc_e2m1_sr.argtypes = [C.c_float, u32]
+        L.orc_e2m1_sr.argtypes = [C.c_float, C.c_uint16]
         L.orc_e4m3_rne_sat.restype = C.c_uint8
         L.orc_e4m3_rne_sat.argtypes = [C.c_float]
         L.orc_floor_log2.restype = C.c_int
@@ -59,10 +60,14 @@ def lib():
         L.orc_draw.argtypes = [u64, u32, u64]
         L.orc_draw_n.restype = None
         L.orc_draw_n.argtypes = [u64, u32, u64, i64, u32p]
+        L.orc_draw16.restype = C.c_uint16
+        L.orc_draw16.argtypes = [u64, u32, u64]
+        L.orc_draw16_n.restype = None
+        L.orc_draw16_n.argtypes = [u64, u32, u64, i64, u16p]
         L.orc_e2m1_rtn_n.restype = None
         L.orc_e2m1_rtn_n.argtypes = [f32p, i64, u8p]
         L.orc_e2m1_sr_n.restype = None
-        L.orc_e2m1_sr_n.argtypes = [f32p, u32p, i64, u8p]
+        L.orc_e2m1_sr_n.argtypes = [f32p, u16p, i64, u8p]
         L.orc_e4m3_rne_sat_n.restype = None
         L.orc_e4m3_rne_sat_n.argtypes = [f32p, i64, u8p]
         L.orc_rht_signs.restype = None
@@ -129,8 +134,11 @@ def e2m1_rtn(v) -> np.ndarray:
 
 
 def e2m1_sr(v, u) -> np.ndarray:
+    """Stochastic E2M1 codes of v with 16-bit draws u (0 .. 65535)."""
     v = _f32(v).reshape(-1)
-    u = np.ascontiguousarray(np.asarray(u, dtype=np.uint32).reshape(-1))
+    u = np.asarray(u)
+    assert u.size == 0 or (u.min() >= 0 and u.max() <= 0xFFFF), "draws are 16-bit"
+    u = np.ascontiguousarray(u.astype(np.uint16).reshape(-1))
     assert u.size == v.size
     out = np.empty(v.size, np.uint8)
     lib().orc_e2m1_sr_n(v, u, v.size, out)
@@ -153,8 +161,16 @@ def philox4x32_10(ctr, key) -> np.ndarray:
 
 
 def draws(seed: int, stream: int, i0: int, n: int) -> np.ndarray:
+    """32-bit draws i0 .. i0 + n - 1 of a stream (word i mod 4 of block i / 4)."""
     out = np.empty(n, np.uint32)
     lib().orc_draw_n(seed, stream, i0, n, out)
+    return out
+
+
+def draws16(seed: int, stream: int, i0: int, n: int) -> np.ndarray:
+    """16-bit stochastic-rounding draws i0 .. i0 + n - 1 of a stream."""
+    out = np.empty(n, np.uint16)
+    lib().orc_draw16_n(seed, stream, i0, n, out)
     return out
 
 

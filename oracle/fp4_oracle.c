@@ -112,12 +112,15 @@ uint8_t orc_e2m1_rtn(float v) {
   return (uint8_t)(best | (signbit(v) ? 8 : 0));
 }
 
-/* Stochastic rounding to E2M1 with one 32-bit uniform draw u.
+/* Stochastic rounding to E2M1 with one 16-bit uniform draw u (0 .. 65535).
  * [FQT] stochastic rounding in the backward and update passes;
  * [FP4] "stochastic rounding of gradients".
- * reading: with lo <= |v| <= hi the neighbouring levels and p = (|v|-lo)/(hi-lo),
- * round up iff u < ceil(p * 2^32); |v| is first clamped to 6. */
-uint8_t orc_e2m1_sr(float v, uint32_t u) {
+ * reading: with lo <= |v| <= hi the neighbouring levels (|v| first clamped to
+ * 6) and p = (|v| - lo) / (hi - lo), round up iff floor(p * 2^16) + u >= 2^16.
+ * Over the 2^16 equally likely draws the value rounds up with probability
+ * floor(p * 2^16) / 2^16: p truncated to 16 bits, so the expected result
+ * lies within (hi - lo) * 2^-16 below |v| (never above it). */
+uint8_t orc_e2m1_sr(float v, uint16_t u) {
   double a = fabs((double)v);
   if (a > 6.0) a = 6.0;
   int lo = 0, hi = 7;
@@ -135,8 +138,8 @@ uint8_t orc_e2m1_sr(float v, uint32_t u) {
   } else {
     double l = orc_e2m1_value((uint8_t)lo), h = orc_e2m1_value((uint8_t)hi);
     double p = (a - l) / (h - l);                 /* exact: power-of-two gap */
-    uint64_t T = (uint64_t)ceil(ldexp(p, 32));    /* exact: p has <= 26 bits */
-    code = ((uint64_t)u < T) ? hi : lo;
+    uint32_t k = (uint32_t)floor(ldexp(p, 16));   /* exact: p has <= 26 bits */
+    code = (k + (uint32_t)u >= 65536u) ? hi : lo;
   }
   return (uint8_t)(code | (signbit(v) ? 8 : 0));
 }
@@ -236,6 +239,14 @@ uint32_t orc_draw(uint64_t seed, uint32_t stream, uint64_t i) {
   uint32_t out[4];
   orc_philox4x32_10(ctr, key, out);
   return out[i & 3];
+}
+
+/* The 16-bit draw of element i of a stream, for stochastic rounding.
+ * reading: the low (i even) or high (i odd) half of the 32-bit draw i / 2,
+ * so one Philox block (counter i / 8) serves eight consecutive elements. */
+uint16_t orc_draw16(uint64_t seed, uint32_t stream, uint64_t i) {
+  uint32_t w = orc_draw(seed, stream, i >> 1);
+  return (uint16_t)((i & 1) ? (w >> 16) : (w & 0xFFFFu));
 }
 
 /* ------------------------------------------------------------------------ */
@@ -346,7 +357,7 @@ static void nvfp4_rows_worker(void* p, int64_t r0, int64_t r1) {
           code = orc_e2m1_rtn(v);
         } else {
           uint64_t idx = (uint64_t)(q->row_offset + r) * (uint64_t)C + (uint64_t)c;
-          code = orc_e2m1_sr(v, orc_draw(q->sr_seed, q->sr_stream, idx));
+          code = orc_e2m1_sr(v, orc_draw16(q->sr_seed, q->sr_stream, idx));
         }
         uint8_t* byte = &q->codes[r * (C / 2) + c / 2];
         if ((c & 1) == 0) *byte = (uint8_t)((*byte & 0xF0) | code);
@@ -479,7 +490,7 @@ static void mxfp4_rows_worker(void* p, int64_t r0, int64_t r1) {
           code = orc_e2m1_rtn(v);
         } else {
           uint64_t idx = (uint64_t)(q->row_offset + r) * (uint64_t)C + (uint64_t)c;
-          code = orc_e2m1_sr(v, orc_draw(q->sr_seed, q->sr_stream, idx));
+          code = orc_e2m1_sr(v, orc_draw16(q->sr_seed, q->sr_stream, idx));
         }
         uint8_t* byte = &q->codes[r * (C / 2) + c / 2];
         if ((c & 1) == 0) *byte = (uint8_t)((*byte & 0xF0) | code);
@@ -533,7 +544,7 @@ void orc_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t R, int6
 void orc_e2m1_rtn_n(const float* v, int64_t n, uint8_t* out) {
   for (int64_t i = 0; i < n; ++i) out[i] = orc_e2m1_rtn(v[i]);
 }
-void orc_e2m1_sr_n(const float* v, const uint32_t* u, int64_t n, uint8_t* out) {
+void orc_e2m1_sr_n(const float* v, const uint16_t* u, int64_t n, uint8_t* out) {
   for (int64_t i = 0; i < n; ++i) out[i] = orc_e2m1_sr(v[i], u[i]);
 }
 void orc_e4m3_rne_sat_n(const float* t, int64_t n, uint8_t* out) {
@@ -541,4 +552,7 @@ void orc_e4m3_rne_sat_n(const float* t, int64_t n, uint8_t* out) {
 }
 void orc_draw_n(uint64_t seed, uint32_t stream, uint64_t i0, int64_t n, uint32_t* out) {
   for (int64_t i = 0; i < n; ++i) out[i] = orc_draw(seed, stream, i0 + (uint64_t)i);
+}
+void orc_draw16_n(uint64_t seed, uint32_t stream, uint64_t i0, int64_t n, uint16_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_draw16(seed, stream, i0 + (uint64_t)i);
 }

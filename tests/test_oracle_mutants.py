@@ -34,9 +34,16 @@ MUTANTS = [
      "double d = fabs(a - orc_e2m1_value((uint8_t)c));\n    if (d <= bestd) {", 0),
     ("e2m1 sign of a negative zero lost", "return (uint8_t)(best | (signbit(v) ? 8 : 0));",
      "return (uint8_t)(best | (v < 0 ? 8 : 0));", 0),
-    ("SR threshold off by one", "code = ((uint64_t)u < T) ? hi : lo;",
-     "code = ((uint64_t)u <= T) ? hi : lo;", 0),
-    ("SR threshold rounded down", "ceil(ldexp(p, 32))", "floor(ldexp(p, 32))", 0),
+    ("SR carry test off by one", "code = (k + (uint32_t)u >= 65536u) ? hi : lo;",
+     "code = (k + (uint32_t)u > 65536u) ? hi : lo;", 0),
+    ("SR fraction rounded up", "(uint32_t)floor(ldexp(p, 16))", "(uint32_t)ceil(ldexp(p, 16))", 0),
+    ("SR fraction to 15 bits", "(uint32_t)floor(ldexp(p, 16))", "(uint32_t)floor(ldexp(p, 15))", 0),
+    ("SR decided on the complemented draw", "code = (k + (uint32_t)u >= 65536u) ? hi : lo;",
+     "code = (k + (uint32_t)(65535u - u) >= 65536u) ? hi : lo;", 0),
+    ("16-bit draw halves swapped", "return (uint16_t)((i & 1) ? (w >> 16) : (w & 0xFFFFu));",
+     "return (uint16_t)((i & 1) ? (w & 0xFFFFu) : (w >> 16));", 0),
+    ("16-bit draw from 32-bit draw i, not i / 2", "uint32_t w = orc_draw(seed, stream, i >> 1);",
+     "uint32_t w = orc_draw(seed, stream, i);", 0),
     ("E4M3 exponent bias", "ldexp(1.0 + (double)m / 8.0, e - 7)",
      "ldexp(1.0 + (double)m / 8.0, e - 8)", 0),
     ("E4M3 saturates to NaN", "if (a > 448.0) return 0x7E;", "if (a > 448.0) return 0x7F;", 0),

@@ -170,7 +170,7 @@ def test_sr_draw_index_is_row_major_in_the_operand(fmt):
     else:
         q = O.mxfp4_quantize(x, "sr", sr_seed=seed, sr_stream=stream, row_offset=off)
         assert np.all(q["scales"] == 127)
-    u = O.draws(seed, stream, off * C, R * C).reshape(R, C)
+    u = O.draws16(seed, stream, off * C, R * C).reshape(R, C)
     want = O.e2m1_sr(x.reshape(-1), u.reshape(-1)).reshape(R, C)
     assert np.array_equal(_codes(q["codes"]), want)
 

@@ -3,8 +3,10 @@
 Stochastic rounding ("FP4 All the Way", Key points: stochastic rounding for
 the backward and update passes) is pinned by what the definition of an
 unbiased stochastic rounding fixes: lattice points are fixed, the rounding
-is unbiased (mean over 4096 seeds within 3 sigma), the up-probability is the
-exact fraction of the gap, and for a fixed draw the result is monotone in v.
+is unbiased (mean over 4096 seeds within 3 sigma; exactly, over all 2^16
+draws, for values whose gap fraction has at most 16 bits), the up-probability
+is the fraction of the gap to 16 bits, and for a fixed draw the result is
+monotone in v.
 Philox is pinned block for block against an independent Philox4x32-10
 (cuRAND's host generator, which runs on the CPU), statistically (uniformity,
 bit balance, independence of streams) and by its counter structure.
@@ -22,37 +24,58 @@ def _val(codes):
 
 
 def test_lattice_points_fixed_for_any_draw():
-    u = np.random.default_rng(0).integers(0, 2**32, 64, dtype=np.uint64).astype(np.uint32)
+    u = np.arange(0, 65536, 1024, dtype=np.uint32).astype(np.uint16)
+    u = np.concatenate([u, np.array([1, 65535], np.uint16)])
     for lv in LEVELS:
         for s in (1.0, -1.0):
-            v = np.full(64, s * lv, np.float32)
+            v = np.full(u.size, s * lv, np.float32)
             out = _val(O.e2m1_sr(v, u))
             assert np.all(out == s * lv)
 
 
-def test_up_probability_is_exact_fraction_of_gap():
-    # v = 1.25 sits at p = 1/2 of the gap [1, 1.5]: up iff u < 2^31
-    v = np.full(4, 1.25, np.float32)
-    u = np.array([0, 2**31 - 1, 2**31, 2**32 - 1], np.uint32)
-    assert list(_val(O.e2m1_sr(v, u))) == [1.5, 1.5, 1.0, 1.0]
-    # v = 2.25 is p = 1/4 of [2, 3]: up iff u < 2^30
-    v = np.full(3, 2.25, np.float32)
-    u = np.array([2**30 - 1, 2**30, 0], np.uint32)
-    assert list(_val(O.e2m1_sr(v, u))) == [3.0, 2.0, 3.0]
-    # v = 5.5 is p = 3/4 of [4, 6]: up iff u < 3 * 2^30
-    v = np.full(2, 5.5, np.float32)
-    u = np.array([3 * 2**30 - 1, 3 * 2**30], np.uint32)
-    assert list(_val(O.e2m1_sr(v, u))) == [6.0, 4.0]
-    # beyond 6 saturates; a tiny positive value rounds up only for u = 0
-    assert list(_val(O.e2m1_sr(np.array([9.0, 1e-30, 1e-30], np.float32),
-                               np.array([0, 0, 1], np.uint32)))) == [6.0, 0.5, 0.0]
+def _up_count(v: float) -> int:
+    """How many of the 2^16 possible draws round |v| up (exhaustive)."""
+    u = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    out = np.abs(_val(O.e2m1_sr(np.full(65536, v, np.float32), u)))
+    a = min(abs(float(v)), 6.0)
+    lo = max(l for l in LEVELS if l <= a)
+    hi = min(l for l in LEVELS if l >= a)
+    assert np.all((out == lo) | (out == hi))
+    return int((out == hi).sum()) if hi != lo else 0
 
 
-def test_extreme_draws_decide_every_interior_value():
-    """Strictly between two levels 0 < p < 1, so ceil(p * 2^32) lies in
-    [1, 2^32 - 1]: the draw 0 always rounds up and the draw 2^32 - 1 never
-    does, down to p of a single binary32 subnormal (a rounded-down threshold
-    would send the smallest p to the lower level with every draw)."""
+def test_exact_up_probability_on_the_16_bit_grid():
+    """Over all 2^16 draws, a value whose gap fraction p has at most 16 bits
+    rounds up exactly p * 2^16 times: the rounding is exactly unbiased there
+    (mean = v), at every gap size and both signs."""
+    cases = [(1.25, 0.5), (2.25, 0.25), (5.5, 0.75), (0.3125, 0.625), (-3.875, 0.875),
+             (1.0 + 2.0 ** -17, 2.0 ** -16), (4.0 + 2.0 ** -15, 2.0 ** -16), (-0.5 - 2.0 ** -17, 2.0 ** -16),
+             (5.999969482421875, 1.0 - 2.0 ** -16)]
+    for v, p in cases:
+        assert _up_count(v) == round(p * 65536), (v, p)
+
+
+def test_up_probability_is_p_truncated_to_16_bits():
+    """For any p the up-count lies in (p * 2^16 - 1, p * 2^16]: the bias is
+    below 2^-16 of the gap and towards the lower level; p below 2^-16 never
+    rounds up; beyond 6 saturates."""
+    rng = np.random.default_rng(3)
+    vals = np.concatenate([rng.uniform(-6, 6, 48), [2.0 ** -20, 1.0 + 2.0 ** -20, 4.0 + 2.0 ** -18]])
+    for v in vals.astype(np.float32):
+        a = abs(float(v))
+        lo = max(l for l in LEVELS if l <= a)
+        hi = min(l for l in LEVELS if l >= a)
+        if hi == lo:
+            continue
+        x = (a - lo) / (hi - lo) * 65536
+        n = _up_count(float(v))
+        assert x - 1 < n <= x, (v, n, x)
+    assert _up_count(9.0) == 0 and abs(_val(O.e2m1_sr(np.float32([9.0]), [0]))[0]) == 6.0
+
+
+def test_extreme_draws():
+    """The draw 0 rounds every interior value down; the draw 2^16 - 1 rounds
+    up exactly the values at least 2^-16 of the gap above the lower level."""
     rng = np.random.default_rng(7)
     v = np.concatenate([rng.uniform(-6.0, 6.0, 4096),
                         2.0 ** -np.arange(2, 150, dtype=np.float64),
@@ -64,17 +87,18 @@ def test_extreme_draws_decide_every_interior_value():
     a = np.abs(v).astype(np.float64)
     hi = np.array([lv[lv > x].min() for x in a])
     lo = np.array([lv[lv < x].max() for x in a])
-    up = np.abs(_val(O.e2m1_sr(v, np.zeros(v.size, np.uint32))))
-    down = np.abs(_val(O.e2m1_sr(v, np.full(v.size, 2**32 - 1, np.uint32))))
-    assert np.array_equal(up, hi)
+    down = np.abs(_val(O.e2m1_sr(v, np.zeros(v.size, np.uint16))))
+    top = np.abs(_val(O.e2m1_sr(v, np.full(v.size, 65535, np.uint16))))
     assert np.array_equal(down, lo)
+    want = np.where((a - lo) / (hi - lo) >= 2.0 ** -16, hi, lo)
+    assert np.array_equal(top, want)
 
 
 def test_monotone_in_v_for_fixed_draw():
     rng = np.random.default_rng(4)
     v = np.sort(rng.uniform(-7, 7, 5000).astype(np.float32))
     for _ in range(8):
-        u = np.full(v.size, rng.integers(0, 2**32, dtype=np.uint64), np.uint32)
+        u = np.full(v.size, rng.integers(0, 2**16), np.uint16)
         out = _val(O.e2m1_sr(v, u))
         assert np.all(np.diff(out) >= 0)
 
@@ -84,7 +108,7 @@ def test_unbiased_over_4096_seeds():
                      -0.6, -2.6, -4.1], np.float32)
     nseed = 4096
     for k, v in enumerate(vals):
-        u = np.array([O.draws(seed, 7, k, 1)[0] for seed in range(nseed)], np.uint32)
+        u = np.array([O.draws16(seed, 7, k, 1)[0] for seed in range(nseed)], np.uint16)
         out = _val(O.e2m1_sr(np.full(nseed, v, np.float32), u))
         a = abs(float(v))
         lo = max(l for l in LEVELS if l <= a)
@@ -92,6 +116,18 @@ def test_unbiased_over_4096_seeds():
         p = (a - lo) / (hi - lo)
         sigma = (hi - lo) * np.sqrt(p * (1 - p) / nseed)
         assert abs(out.mean() - float(v)) <= 3 * sigma, (v, out.mean(), sigma)
+
+
+def test_16_bit_draws_are_halves_of_the_32_bit_draws():
+    """Draw i of the 16-bit stochastic-rounding stream is the low (i even) or
+    high (i odd) half of the 32-bit draw i / 2, which the known answers
+    below pin to an independent Philox4x32-10: one Philox block gives the
+    draws of eight consecutive elements."""
+    for seed, stream, i0 in ((0, 0, 0), (0x0123456789ABCDEF, 3, 8 * 12345), (2**64 - 1, 2, 2**35)):
+        d32 = O.draws(seed, stream, i0 // 2, 64)
+        d16 = O.draws16(seed, stream, i0, 128)
+        want = np.stack([d32 & 0xFFFF, d32 >> 16], axis=1).reshape(-1)
+        assert np.array_equal(d16.astype(np.uint32), want)
 
 
 def test_philox_structure_and_determinism():
