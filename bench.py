@@ -630,10 +630,11 @@ def run_swiglu(device, layers=8, hidden=2048, ffn=8192, tokens=16384, seed=0, ch
         h = torch.empty((M, H), dtype=torch.bfloat16, device=device)
         F.fqt_linear_fwd(cfg, a, w_d[l], h, sv_d[l], ws)
         acts.append(h)
-    d, dxs, dwg, dwd, dys = dy_top, [None] * L, [None] * L, [None] * L, {}
+    d, dxs, dwg, dwd, dys, das = dy_top, [None] * L, [None] * L, [None] * L, {}, [None] * L
     for l in reversed(range(L)):
         dys[(l, "d")] = d
         da = torch.empty((M, Fd), dtype=torch.bfloat16, device=device)
+        das[l] = da
         dwd[l] = torch.empty((H, Fd), dtype=torch.float32, device=device)
         F.fqt_linear_bwd(cfg, d, sv_d[l], da, dwd[l], ws)
         g, u = gus[l][:, :Fd], gus[l][:, Fd:]
@@ -697,6 +698,43 @@ def run_swiglu(device, layers=8, hidden=2048, ffn=8192, tokens=16384, seed=0, ch
     def rel(a, b):
         return float((a.float() - b).norm() / b.norm())
 
+    # ---- per-layer local check: each linear's Y, dX and dW against FP32
+    # products of THAT linear's own inputs in the quantized stack (its BF16
+    # input activation and incoming gradient), so that the comparison does not
+    # depend on the errors the layers below or above carried in.  The bound
+    # comes from the quantization noise of the operands themselves: with
+    # relative noise r_a, r_b (||q(a) - a|| / ||a||, from fp4_quant_noise) a
+    # product's relative error is about sqrt(r_a^2 + r_b^2); twice that is
+    # allowed.  A wrong or missing gradient has a relative error near 1.
+    def nsr(x, q):
+        F.fp4_quant_noise(x, q, sums, ws)
+        sx, sn = sums.tolist()
+        return (sn / sx) ** 0.5 if sx > 0 else 0.0
+
+    local = []
+    prev_tf32 = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = False
+    try:
+        for l in range(L):
+            for key, sv, xin, w, y, dyin, dx, dw in (
+                    ("gate_up", sv_gu[l], hin[2 * l], w_gu[l], gus[l], dys[(l, "gu")], dxs[l],
+                     dwg[l]),
+                    ("down", sv_d[l], hin[2 * l + 1], w_d[l], acts[l], dys[(l, "d")], das[l],
+                     dwd[l])):
+                xf, wf, gf = xin.float(), w.float(), dyin.float()
+                r_x, r_w, r_g = nsr(xin, sv.xq), nsr(w, sv.wq), nsr(dyin, sv.dyq)
+                r_xt = nsr(xin.t().contiguous(), sv.xq_t)
+                r_wt = nsr(w.t().contiguous(), sv.wq_t)
+                r_gt = nsr(dyin.t().contiguous(), sv.dyq_t)
+                e = {"y": rel(y, xf @ wf.t()), "dx": rel(dx, gf @ wf), "dw": rel(dw, gf.t() @ xf)}
+                b = {"y": (r_x ** 2 + r_w ** 2) ** 0.5, "dx": (r_g ** 2 + r_wt ** 2) ** 0.5,
+                     "dw": (r_gt ** 2 + r_xt ** 2) ** 0.5}
+                local.append({"layer": l + 1, "linear": key,
+                              **{f"{k}_local": round(v, 5) for k, v in e.items()},
+                              **{f"{k}_noise": round(v, 5) for k, v in b.items()}})
+    finally:
+        torch.backends.cuda.matmul.allow_tf32 = prev_tf32
+
     per_layer = [{"layer": l + 1, "act": round(rel(acts[l], racts[l]), 5),
                   "act_bf16_only": round(rel(bacts[l], racts[l]), 5),
                   "dx": round(rel(dxs[l], rdx[l]), 5),
@@ -729,7 +767,7 @@ def run_swiglu(device, layers=8, hidden=2048, ffn=8192, tokens=16384, seed=0, ch
     return {"case": "swiglu", "layers": L, "hidden": H, "ffn": Fd, "tokens": M,
             "ms_quantized_fwd_bwd": round(ms, 3),
             "tflops_gemm_equiv": round(L * 6 * M * (2 * Fd * H + H * Fd) / (ms * 1e-3) / 1e12, 1),
-            "rel_err_vs_fp32": per_layer, "oracle_rows_checked": checked,
+            "rel_err_vs_fp32": per_layer, "local": local, "oracle_rows_checked": checked,
             "oracle_mismatches": mism}
 
 

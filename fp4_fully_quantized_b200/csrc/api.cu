@@ -276,9 +276,11 @@ fp4_status fp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
   return quantize_impl(x, rows, cols, ld, p, out, out_t, ws, ws_bytes, stream, false);
 }
 
-// The GEMM kernel numbers its 128 x 256 output tiles with 32-bit integers.
+// The GEMM kernel numbers its 128 x 256 output tiles with 32-bit integers and
+// steps through them by the grid size (at most a few thousand CTAs): with at
+// most 2^30 tiles, tile + gridDim.x never overflows.
 static bool gemm_tiles_fit(int64_t M, int64_t N) {
-  return (M / 128) * ((N + 255) / 256) <= (int64_t)INT32_MAX;
+  return (M / 128) * ((N + 255) / 256) <= (int64_t)1 << 30;
 }
 
 // fp4_gemm; with `dry` it only validates the arguments.

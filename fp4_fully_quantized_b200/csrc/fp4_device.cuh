@@ -130,27 +130,44 @@ __device__ __forceinline__ uint32_t e2m1x8_rn(const float* v) {
   return out;
 }
 
-// E2M1 stochastic rounding of one value with draw u: with lo <= |v| <= hi the
-// neighbouring levels (|v| clamped to 6), round up iff u < ceil(p * 2^32),
-// p = (|v| - lo) / (hi - lo).  Returns the 4-bit code (sign kept, also for
-// results of 0).
+// E2M1 stochastic rounding with 16-bit draws: with lo <= |v| <= hi the
+// neighbouring levels (|v| clamped to 6) and p = (|v| - lo) / (hi - lo),
+// round up iff floor(p * 2^16) + u >= 2^16.
 //
-// Branch-free, with the level and the threshold computed together as the two
-// halves of one 64-bit integer (high word: lower level index, low word:
-// ceil(p * 2^32)).  For |v| >= 1 the grid splits each binade of binary32 in
-// two (gaps 0.5, 1, 2), so the lower level is (exponent, top mantissa bit) =
-// bits >> 22, less 252, and ceil(p * 2^32) is the remaining 22 mantissa bits,
-// bits << 10: both halves of bits * 2^10 - 252 * 2^32.  For |v| < 1 the gap is
-// 0.5 everywhere and ceil(|v| * 2^33) (exact: the product is a float below
-// 2^33) has the level (0 or 1) above bit 32 and ceil(p * 2^32) below it.
-__device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t u) {
-  const float a = fminf(fabsf(v), 6.0f);
-  const uint32_t ab = __float_as_uint(a);
-  const uint64_t w_big = (uint64_t)ab * 1024u + 0xFFFFFF0400000000ull;
-  const uint64_t w_small = __float2ull_ru(__fmul_rn(a, 8589934592.0f));   // 2^33
-  const uint64_t w = ab >= 0x3F800000u ? w_big : w_small;
-  const uint32_t level = (uint32_t)(w >> 32) + ((uint32_t)w > u ? 1u : 0u);
-  return level + ((__float_as_uint(v) >> 31) << 3);
+// Branch-free.  code(lo) * 2^16 + p * 2^16 is a concave piecewise-linear map
+// of a = |v|: slope 2^16 / gap for the gaps 0.5 (a < 2), 1 (2 <= a < 4) and
+// 2 (4 <= a <= 6), equal to k * 2^16 at the k-th level, flat from 6 on:
+//   f(a) = min(a * 2^17, (a + 2) * 2^16, (a + 8) * 2^15, 7 * 2^16).
+// The floor of each line is one FMA rounded toward -inf with 2^23 added (in
+// [2^23, 2^24) every float is an integer), and the floor of the min is the
+// min of the floors.  So min(...) as an integer is 2^23 + code(lo) * 2^16 +
+// floor(p * 2^16), below 2^23 + 2^19; adding the draw carries into bit 16
+// exactly when the value rounds up, and bits 16..18 are the code.  NaN
+// inputs give 6 (fminf drops NaN); they are flagged by the amax check.
+__device__ __forceinline__ uint32_t e2m1_sr16_magnitude_bits(float v, uint32_t u16) {
+  const float a = fabsf(v);
+  const float g1 = __fmaf_rd(a, 131072.0f, 8388608.0f);               // a*2^17 + 2^23
+  const float g2 = __fmaf_rd(a, 65536.0f, 8519680.0f);                // (a+2)*2^16 + 2^23
+  const float g3 = __fmaf_rd(a, 32768.0f, 8650752.0f);                // (a+8)*2^15 + 2^23
+  const float m = fminf(fminf(g1, g2), fminf(g3, 8847360.0f));       // 7*2^16 + 2^23
+  return __float_as_uint(m) + u16;                                   // code in bits 16..18
+}
+
+// Eight values -> eight stochastically rounded codes, element j in bits
+// 4j..4j+3 (sign kept, also for results of 0), with the 16-bit draws of one
+// Philox block: element j uses the low (j even) or high (j odd) half of
+// word j / 2.
+__device__ __forceinline__ uint32_t e2m1x8_sr(const float* v, const U4& w) {
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+  uint32_t out = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t u16 = (j & 1) ? (ws[j >> 1] >> 16) : (ws[j >> 1] & 0xFFFFu);
+    const uint32_t t = e2m1_sr16_magnitude_bits(v[j], u16);
+    const uint32_t nib = ((t >> 16) & 7u) | ((__float_as_uint(v[j]) >> 28) & 8u);
+    out |= nib << (4 * j);
+  }
+  return out;
 }
 
 // ---------------------------------------------------------------------------

@@ -444,7 +444,7 @@ bool codes_map(CUtensorMap* m, const uint8_t* codes, int64_t rows, int64_t K, ui
 
 }  // namespace
 
-fp4_status gemm_launch_sfst(const GemmArgs& g, cudaStream_t s) {
+fp4_status gemm_launch(const GemmArgs& g, cudaStream_t s) {
   const bool nv = g.fmt == FP4_NVFP4;
   CUtensorMap ta, tb;
   if (!codes_map(&ta, g.a_codes, g.M, g.K, BM)) return FP4_ERR_CUDA;

@@ -79,7 +79,7 @@ struct Quant2DArgs {
 };
 cudaError_t launch_quant_2d(const Quant2DArgs& a, cudaStream_t s);
 
-// --- GEMM (gemm.cu -> gemm_sfst.cu) ---------------------------------------
+// --- GEMM (gemm_sfst.cu) ----------------------------------------------------
 struct GemmArgs {
   const uint8_t* a_codes; const uint8_t* a_sf; const float* a_sdec;
   const uint8_t* b_codes; const uint8_t* b_sf; const float* b_sdec;
@@ -97,7 +97,5 @@ fp4_status gemm_launch(const GemmArgs& g, cudaStream_t s);
 // Every argument check of fp4_gemm, with nothing enqueued (api.cu).
 fp4_status gemm_validate(const fp4_qtensor* a, const fp4_qtensor* b, const void* c, int64_t ldc,
                          int32_t out_dtype, const void* ws, size_t ws_bytes);
-// Scale factors staged into TMEM by tcgen05.st warps (gemm_sfst.cu).
-fp4_status gemm_launch_sfst(const GemmArgs& g, cudaStream_t s);
 
 }  // namespace fp4impl

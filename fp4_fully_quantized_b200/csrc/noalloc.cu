@@ -12,6 +12,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstdlib>
 #include <mutex>
 
 #include "fp4.h"
@@ -26,26 +27,40 @@ static_assert(FP4_NOALLOC_SCRATCH_BYTES == kNoAllocScratchBytes, "header and lib
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
-struct DeviceScratch {
-  std::once_flag once;
-  void* ptr = nullptr;
-  cudaError_t err = cudaSuccess;
-};
 constexpr int kMaxDevices = 64;
-DeviceScratch g_scratch[kMaxDevices];
+std::mutex g_lookup_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};   // device address once a lookup succeeded
+
+// Host-side fault injection for the failure path of the lookup: the first
+// FP4_NOALLOC_FAIL_LOOKUPS lookups of the process report cudaErrorNotReady
+// instead of calling cudaGetSymbolAddress (read once; unset means 0).
+int injected_failures_left() {
+  static int left = [] {
+    const char* s = std::getenv("FP4_NOALLOC_FAIL_LOOKUPS");
+    return s ? std::atoi(s) : 0;
+  }();
+  return left > 0 ? left-- : 0;
+}
 
 // Device address of the scratch array on the current device.  In host code
 // the array's name is only a host-side stand-in, so the address comes from
-// cudaGetSymbolAddress, once per device, with that device current.
+// cudaGetSymbolAddress, with that device current.  Only a successful lookup
+// is kept: a failed one (a call made during stream capture, a context not yet
+// usable, an error left pending by unrelated work) is retried by the next call
+// and its CUDA error is returned to this one as FP4_ERR_CUDA.
 fp4_status scratch_for_current_device(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FP4_ERR_CUDA;
-  DeviceScratch& d = g_scratch[dev];
-  std::call_once(d.once, [&d] {
-    d.err = cudaGetSymbolAddress(&d.ptr, g_noalloc_scratch);
-  });
-  if (d.err != cudaSuccess || d.ptr == nullptr) return FP4_ERR_CUDA;
-  *out = d.ptr;
+  std::lock_guard<std::mutex> lock(g_lookup_mutex);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = injected_failures_left() > 0
+                              ? cudaErrorNotReady
+                              : cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) return FP4_ERR_CUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
   return FP4_OK;
 }
 

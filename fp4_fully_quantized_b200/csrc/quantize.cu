@@ -292,13 +292,9 @@ quant_rows_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t col
       if constexpr (!SR) {
         packed = e2m1x8_rn(v);
       } else {
+        // one Philox block: the 16-bit draws of these 8 elements
         const uint64_t i0 = (uint64_t)r * (uint64_t)cols + (uint64_t)(c * 8);
-        const U4 w0 = philox_keyed(i0 >> 2, sr_stream, K);
-        const U4 w1 = philox_keyed((i0 >> 2) + 1, sr_stream, K);
-        const uint32_t ud[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-        packed = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) packed += e2m1_sr(v[i], ud[i]) << (4 * i);
+        packed = e2m1x8_sr(v, philox_keyed(i0 >> 3, sr_stream, K));
       }
       if (c < cpr) {
         *reinterpret_cast<uint32_t*>(codes + r * (cols >> 1) + c * 4) = packed;
@@ -430,15 +426,10 @@ quant_cols_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t col
 #pragma unroll
         for (int q = 0; q < 4; ++q) packed[q] = e2m1x8_rn(&v[8 * q]);
       } else {
-        const uint64_t i0 = (uint64_t)k * (uint64_t)rows + (uint64_t)mrow0;
+        const uint64_t i0 = (uint64_t)k * (uint64_t)rows + (uint64_t)mrow0;   // a multiple of 16
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const U4 w = philox4x32_10((i0 >> 2) + q, sr_stream, sr_seed);
-          const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            packed[q >> 1] |= e2m1_sr(v[4 * q + i], u[i]) << (4 * ((4 * q + i) & 7));
-        }
+        for (int q = 0; q < 4; ++q)
+          packed[q] = e2m1x8_sr(&v[8 * q], philox4x32_10((i0 >> 3) + q, sr_stream, sr_seed));
       }
       uint8_t* dst = codes + k * (rows >> 1) + (mrow0 >> 1);
       *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
@@ -575,9 +566,12 @@ quant_2d_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols,
 //   row phase   warp w takes rows w, w + 8, ...; lane l the 8 values at columns
 //               8l .. 8l + 7 (blocks of 16/32 = 2/4 adjacent lanes, Hadamard
 //               stages across lanes by shuffles), 4 code bytes per lane;
-//   column phase thread t takes column t, the tile's 64 rows block by block
-//               down the column, and writes its 32 code bytes and 4 (2)
-//               scale bytes of the transposed operand in one go.
+//   column phase thread t takes columns 2p, 2p + 1 (p = t % 128) over the
+//               tile's rows 32h .. 32h + 31 (h = t / 128), block by block
+//               down the columns, and writes each column's 16 code bytes and
+//               2 (1) scale bytes of the transposed operand in one go.
+// Stochastic rounding draws 16 bits per element: one Philox block serves
+// eight consecutive elements of an output's logical layout.
 // ---------------------------------------------------------------------------
 constexpr int kDualTM = 64, kDualTK = 256, kDualThreads = 256;
 #ifndef FP4_DUAL_CTAS_PER_SM
@@ -608,8 +602,11 @@ __device__ __forceinline__ void block_scale(float bmax, float s_enc, const float
   }
 }
 
+template <int BS>
+constexpr int dual_ctas_per_sm() { return BS == 16 ? kDualCtasPerSm : 2; }
+
 template <int BS, int RHT_R, int RHT_C, bool SR_R, bool SR_C>
-__global__ void __launch_bounds__(kDualThreads, kDualCtasPerSm)
+__global__ void __launch_bounds__(kDualThreads, dual_ctas_per_sm<BS>())
 quant_dual_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
                   uint32_t mask_r, uint32_t mask_c, const __grid_constant__ PhiloxKeys K,
                   uint32_t stream_r,
@@ -703,13 +700,8 @@ quant_dual_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t col
       if constexpr (!SR_R) {
         packed = e2m1x8_rn(v);
       } else {
-        const uint64_t i0 = (uint64_t)r * (uint64_t)cols + (uint64_t)c;
-        const U4 w0 = philox_keyed(i0 >> 2, stream_r, K);
-        const U4 w1 = philox_keyed((i0 >> 2) + 1, stream_r, K);
-        const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-        packed = 0;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) packed |= e2m1_sr(v[q], u[q]) << (4 * q);
+        const uint64_t i0 = (uint64_t)r * (uint64_t)cols + (uint64_t)c;      // a multiple of 8
+        packed = e2m1x8_sr(v, philox_keyed(i0 >> 3, stream_r, K));
       }
       if (active) {
         *reinterpret_cast<uint32_t*>(codes_r + r * (cols >> 1) + (c >> 1)) = packed;
@@ -722,95 +714,106 @@ quant_dual_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t col
     }
 
     // ---------------- column phase (blocks along x's columns) -----------
-    // Thread t encodes column k0 + t over the tile's 64 rows (64/BS blocks),
-    // keeps the 32 code bytes and the block scales in registers and writes
-    // each with as few stores as alignment allows.
-    const int64_t k = k0 + t;
-    if (k < cols) {
-      constexpr int NB = kDualTM / BS;                 // blocks per column in a tile
-      uint32_t cw[kDualTM / 8];                        // packed codes, 8 per word
-      uint32_t sfw = 0;                                // scale byte of block b at 8b
+    // Thread t encodes the column pair k0 + 2p, k0 + 2p + 1 (p = t % 128)
+    // over the tile's rows 32h .. 32h + 31 (h = t / 128): one 32-bit shared
+    // load per row gives both columns (a warp reads 128 contiguous bytes); the
+    // 16 code bytes and the 32 / BS block scales of each column are written
+    // with as few stores as alignment allows.
+    {
+      const int p = t & 127, h = t >> 7;
+      const int64_t kc = k0 + 2 * p;                    // cols % 8 == 0: kc + 1 < cols too
+      const int64_t mh = m0 + 32 * h;                   // first x row of this half
+      if (kc < cols && mh < rows) {
+        constexpr int NB = 32 / BS;                     // blocks per column in a half
+        uint32_t cw[2][4];                              // codes, 8 per word, per column
+        uint32_t sfw[2] = {0u, 0u};                     // scale byte of block b at 8b
 #pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        const int64_t mrow0 = m0 + BS * b;
+        for (int b = 0; b < NB; ++b) {
+          const int tr0 = 32 * h + BS * b;              // first tile row of the block
+          const int64_t mrow0 = m0 + tr0;
+          if (mrow0 >= rows) {                          // rows % BS == 0: whole block out
 #pragma unroll
-        for (int w = 0; w < BS / 8; ++w) cw[b * (BS / 8) + w] = 0;
-        if (mrow0 >= rows) continue;
-        float v[BS];
+            for (int e = 0; e < 2; ++e)
 #pragma unroll
-        for (int q = 0; q < BS; ++q) v[q] = __bfloat162float(tile[buf][BS * b + q][t]);
-        if constexpr (RHT_C > 0) {
+              for (int w = 0; w < BS / 8; ++w) cw[e][b * (BS / 8) + w] = 0u;
+            continue;
+          }
+          uint32_t raw[BS];
 #pragma unroll
-          for (int q = 0; q < RHT_C; ++q)
-            if ((mask_c >> q) & 1u) v[q] = -v[q];
+          for (int q = 0; q < BS; ++q)
+            raw[q] = *reinterpret_cast<const uint32_t*>(&tile[buf][tr0 + q][2 * p]);
 #pragma unroll
-          for (int hh = 1; hh < RHT_C; hh <<= 1) {
+          for (int e = 0; e < 2; ++e) {
+            float v[BS];
 #pragma unroll
-            for (int q = 0; q < RHT_C; ++q) {
-              if (q & hh) continue;
-              const float x0 = v[q], x1 = v[q + hh];
-              v[q] = __fadd_rn(x0, x1);
-              v[q + hh] = __fsub_rn(x0, x1);
+            for (int q = 0; q < BS; ++q)
+              v[q] = __uint_as_float(e ? (raw[q] & 0xFFFF0000u) : (raw[q] << 16));
+            if constexpr (RHT_C > 0) {
+#pragma unroll
+              for (int q = 0; q < RHT_C; ++q)
+                if ((mask_c >> q) & 1u) v[q] = -v[q];
+#pragma unroll
+              for (int hh = 1; hh < RHT_C; hh <<= 1) {
+#pragma unroll
+                for (int q = 0; q < RHT_C; ++q) {
+                  if (q & hh) continue;
+                  const float x0 = v[q], x1 = v[q + hh];
+                  v[q] = __fadd_rn(x0, x1);
+                  v[q + hh] = __fsub_rn(x0, x1);
+                }
+              }
+              const float cn = rht_scale<RHT_C>();
+#pragma unroll
+              for (int q = 0; q < RHT_C; ++q) v[q] = __fmul_rn(v[q], cn);
+            }
+            float bmax = 0.0f;
+#pragma unroll
+            for (int q = 0; q < BS; ++q) bmax = fmaxf(bmax, fabsf(v[q]));
+            uint32_t sf;
+            float inv;
+            block_scale<NV>(bmax, se_c, inv_tab[1], sf, inv);
+            sfw[e] |= sf << (8 * b);
+#pragma unroll
+            for (int q = 0; q < BS; ++q) v[q] = __fmul_rn(v[q], inv);
+            if constexpr (!SR_C) {
+#pragma unroll
+              for (int w = 0; w < BS / 8; ++w) cw[e][b * (BS / 8) + w] = e2m1x8_rn(&v[8 * w]);
+            } else {
+              // element (kc + e, mrow0 + q) of x^T: draw index (kc + e) * rows + mrow0 + q,
+              // a multiple of 8 at q = 0
+              const uint64_t i0 = (uint64_t)(kc + e) * (uint64_t)rows + (uint64_t)mrow0;
+#pragma unroll
+              for (int w = 0; w < BS / 8; ++w)
+                cw[e][b * (BS / 8) + w] = e2m1x8_sr(&v[8 * w], philox_keyed((i0 >> 3) + w, stream_c, K));
             }
           }
-          const float cn = rht_scale<RHT_C>();
-#pragma unroll
-          for (int q = 0; q < RHT_C; ++q) v[q] = __fmul_rn(v[q], cn);
         }
-        float bmax = 0.0f;
+        const int64_t left = rows - mh;                 // valid rows in this half (> 0)
+        const int nvalid = left >= 32 ? NB : (int)(left / BS);
+        const int64_t sb0 = mh / BS;                    // first block of this half
 #pragma unroll
-        for (int q = 0; q < BS; ++q) bmax = fmaxf(bmax, fabsf(v[q]));
-        uint32_t sf;
-        float inv;
-        block_scale<NV>(bmax, se_c, inv_tab[1], sf, inv);
-        sfw |= sf << (8 * b);
-#pragma unroll
-        for (int q = 0; q < BS; ++q) v[q] = __fmul_rn(v[q], inv);
-        if constexpr (!SR_C) {
-#pragma unroll
-          for (int w = 0; w < BS / 8; ++w) cw[b * (BS / 8) + w] = e2m1x8_rn(&v[8 * w]);
-        } else {
-          const uint64_t i0 = (uint64_t)k * (uint64_t)rows + (uint64_t)mrow0;
-#pragma unroll
-          for (int q = 0; q < BS / 4; ++q) {
-            const U4 d = philox_keyed((i0 >> 2) + q, stream_c, K);
-            const uint32_t u[4] = {d.x, d.y, d.z, d.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              cw[b * (BS / 8) + (q >> 1)] += e2m1_sr(v[4 * q + e], u[e]) << (4 * ((4 * q + e) & 7));
+        for (int e = 0; e < 2; ++e) {
+          const int64_t k = kc + e;
+          uint8_t* dst = codes_c + k * (rows >> 1) + (mh >> 1);
+          if (nvalid == NB && ((rows >> 1) & 15) == 0) {  // 16-byte aligned row of x^T
+            *reinterpret_cast<uint4*>(dst) = make_uint4(cw[e][0], cw[e][1], cw[e][2], cw[e][3]);
+          } else {                                         // rows % 16 == 0: 8-byte aligned
+            *reinterpret_cast<uint2*>(dst) = make_uint2(cw[e][0], cw[e][1]);
+            if (left > 16) *reinterpret_cast<uint2*>(dst + 8) = make_uint2(cw[e][2], cw[e][3]);
           }
-        }
-      }
-      const int64_t sb0 = m0 / BS;                     // first block of the tile
-      const int64_t left = (rows - m0) / BS;           // rows % BS == 0
-      const int nvalid = left < NB ? (int)left : NB;
-      uint8_t* dst = codes_c + k * (rows >> 1) + (m0 >> 1);
-      if (nvalid == NB && ((rows >> 1) & 15) == 0) {   // 16-byte aligned row of x^T
-        *reinterpret_cast<uint4*>(dst) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-        *reinterpret_cast<uint4*>(dst + 16) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
-      } else {                                         // rows % 16 == 0: 8-byte aligned
-#pragma unroll
-        for (int h = 0; h < kDualTM / 16; ++h)
-          if (16 * h < rows - m0) *reinterpret_cast<uint2*>(dst + 8 * h) = make_uint2(cw[2 * h], cw[2 * h + 1]);
-      }
-      if (scales_c != nullptr) {
-        uint8_t* sd = scales_c + k * S_c + sb0;
-        if (nvalid == NB && (S_c % NB) == 0 && (reinterpret_cast<uintptr_t>(scales_c) % NB) == 0) {
-          if constexpr (NB == 4) *reinterpret_cast<uint32_t*>(sd) = sfw;
-          else *reinterpret_cast<uint16_t*>(sd) = (uint16_t)sfw;
-        } else {
-          for (int b = 0; b < nvalid; ++b) sd[b] = (uint8_t)(sfw >> (8 * b));
-        }
-      }
-      if (mma_c != nullptr) {
-        // blocks sb0 .. sb0 + NB - 1 share one 4-byte slot group (sb0 % 4 == 0
-        // for NVFP4, sb0 % 2 == 0 for MXFP4): contiguous and aligned
-        uint8_t* md = mma_c + mma_sf_offset(k, sb0, S_c4);
-        if (nvalid == NB && (reinterpret_cast<uintptr_t>(mma_c) % NB) == 0) {
-          if constexpr (NB == 4) *reinterpret_cast<uint32_t*>(md) = sfw;
-          else *reinterpret_cast<uint16_t*>(md) = (uint16_t)sfw;
-        } else {
-          for (int b = 0; b < nvalid; ++b) md[b] = (uint8_t)(sfw >> (8 * b));
+          if (scales_c != nullptr) {
+            uint8_t* sd = scales_c + k * S_c + sb0;
+            if (NB == 2 && nvalid == 2 && (reinterpret_cast<uintptr_t>(sd) & 1) == 0)
+              *reinterpret_cast<uint16_t*>(sd) = (uint16_t)sfw[e];
+            else
+              for (int b = 0; b < nvalid; ++b) sd[b] = (uint8_t)(sfw[e] >> (8 * b));
+          }
+          if (mma_c != nullptr) {
+            // NVFP4: sb0 % 4 is 0 or 2, so both bytes share one 4-byte slot group
+            uint8_t* md = mma_c + mma_sf_offset(k, sb0, S_c4);
+            if (NB == 2 && nvalid == 2) *reinterpret_cast<uint16_t*>(md) = (uint16_t)sfw[e];
+            else for (int b = 0; b < nvalid; ++b) md[b] = (uint8_t)(sfw[e] >> (8 * b));
+          }
         }
       }
     }
@@ -926,7 +929,7 @@ static cudaError_t dual_variant(const DualQuantArgs& a, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDualSmem);
   if (e != cudaSuccess) return e;
   const int64_t ntiles = ((a.rows + kDualTM - 1) / kDualTM) * ((a.cols + kDualTK - 1) / kDualTK);
-  const int grid = grid_for(ntiles, 1, kDualCtasPerSm);
+  const int grid = grid_for(ntiles, 1, dual_ctas_per_sm<BS>());
   kern<<<grid, kDualThreads, kDualSmem, s>>>(
       static_cast<const __nv_bfloat16*>(a.x), a.rows, a.cols, a.ld, a.mask_r, a.mask_c,
       philox_keys(a.sr_seed), a.stream_r, a.stream_c, a.amax_src_r, a.amax_src_c, a.amax_out_r,

@@ -260,9 +260,10 @@ fp4_status fqt_linear_bwd(const fqt_linear_cfg* cfg, int64_t M, int64_t N, int64
  *   - Problems whose workspace need (fp4_workspace_bytes(M, N, K)) exceeds
  *     FP4_NOALLOC_SCRATCH_BYTES are rejected with FP4_ERR_WORKSPACE.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
- *   - The first call on a device looks up the array's device address (once
- *     per device, with that device current); make that first call before any
- *     stream capture.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and keeps it for the rest of the process; make
+ *     that first call before any stream capture.  A lookup that fails returns
+ *     FP4_ERR_CUDA, keeps nothing, and is tried again by the next call.
  *   - Every call shares the one array: each call clears its status block on
  *     `stream` first, and calls that overlap on the GPU (other streams, other
  *     threads) race on it.  Device conditions of a call are not reported

@@ -179,3 +179,7 @@ def test_gemm_rejects_tile_counts_beyond_32_bits(lib):
     amax = C.c_void_p(1 << 23)
     assert lib.fp4_gemm_quant(C.byref(a), C.byref(b), 1.0, amax, C.byref(out), None, ws, 256,
                               None) == 2
+    # just above the limit of 2^30 tiles: 2^23 row blocks x (2^7 + 1) column blocks
+    b2 = _q((1 << 15) + 256, 128)
+    assert lib.fp4_gemm(C.byref(a), C.byref(b2), 1.0, c, (1 << 15) + 256, 0, None, ws, 256,
+                        None) == 2

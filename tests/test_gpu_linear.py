@@ -85,7 +85,7 @@ def _compare_ops(F, sv, ops, cfg):
         assert float(t.s_dec.item()) == float(ref["s_dec"]), name
 
 
-@pytest.mark.parametrize("variant", ["nvfp4", "nvfp4_wgrad_rht", "mxfp4"])
+@pytest.mark.parametrize("variant", ["nvfp4", "nvfp4_wgrad_rht", "nvfp4_1d_rht_all", "mxfp4"])
 def test_tiny_linear_layer(gpu_lib, variant):
     F = gpu_lib
     d = S.tiny_linear(seed=0)
@@ -93,6 +93,11 @@ def test_tiny_linear_layer(gpu_lib, variant):
     cfg = F.linear_cfg(fmt, out_dtype=F.OUT_F32)
     if variant == "nvfp4_wgrad_rht":
         cfg.rht_mask = F.RHT_WGRAD
+    if variant == "nvfp4_1d_rht_all":
+        # 1x16 weights, so that fprop and dgrad can rotate too: every operand
+        # of the three GEMMs goes through the 16-point transform
+        cfg.w_block = F.BLOCK_1D
+        cfg.rht_mask = F.RHT_FPROP | F.RHT_DGRAD | F.RHT_WGRAD
     X, W, dY = d["X"], d["W"], d["dY"]
     sv, y, dx, dw = _run_layer(F, X, W, dY, cfg)
     ops, ry, rdx, rdw = _oracle_layer(S.as_f32(X), S.as_f32(W), S.as_f32(dY), cfg)

@@ -99,6 +99,24 @@ def test_nvfp4_row_and_transposed_together(gpu_lib, shape):
                                       sr_seed=0, sr_stream=3), 0)
 
 
+@pytest.mark.parametrize("shape", [(128, 256), (48, 80), (1024, 512), (64, 272)])
+@pytest.mark.parametrize("rht_t", [0, 16])
+@pytest.mark.parametrize("rnd,rnd_t", [(RTN, RTN), (RTN, SR), (SR, RTN), (SR, SR)])
+def test_nvfp4_dual_with_rotated_rows(gpu_lib, shape, rht_t, rnd, rnd_t):
+    """The fused row-wise + transposed NVFP4 quantizer with the 16-point
+    Hadamard transform on the row-wise output (and with or without it on the
+    transposed one), every pair of roundings: both outputs bit-exact."""
+    F = gpu_lib
+    x, _ = S.outlier_columns(*shape, seed=5)
+    q, qt = _gpu_quant(F, x, 0, round=rnd, round_t=rnd_t, rht_n=16, rht_n_t=rht_t, seed=9,
+                       stream=1, stream_t=2, col=True)
+    xf = S.as_f32(x)
+    m = lambda r: "sr" if r == SR else "rtn"
+    _check_1d(q, O.nvfp4_quantize_1d(xf, m(rnd), rht_n=16, rht_seed=9, sr_seed=9, sr_stream=1), 0)
+    _check_1d(qt, O.nvfp4_quantize_1d(np.ascontiguousarray(xf.T), m(rnd_t), rht_n=rht_t,
+                                      rht_seed=9, sr_seed=9, sr_stream=2), 0)
+
+
 @pytest.mark.parametrize("shape", [(256, 256), (48, 96), (4096, 512)])
 def test_nvfp4_2d(gpu_lib, shape):
     F = gpu_lib

@@ -1,11 +1,22 @@
 """Chained SwiGLU MLP stack (8 layers, hidden 2048, FFN 8192, 16384 tokens):
 NVFP4 forward through every layer, SR gradients back, each linear through
-fqt_linear_fwd / fqt_linear_bwd.  Checks: sampled rows of the first and last
-layers' quantized operands are bit-exact with the oracle; every error against
-the unquantized FP32 stack is finite; the first layer's activations carry
-NVFP4-sized noise (a relative error of at most 0.3: E2M1 round-to-nearest is
-off by at most a quarter of a value above the block's smallest level, and the
-GEMM averages that over the contraction); no layer diverges (all < 2)."""
+fqt_linear_fwd / fqt_linear_bwd.
+
+Checks:
+  * sampled rows of the first and last layers' quantized operands are
+    bit-exact with the oracle;
+  * every linear of every layer, on its own inputs in the quantized stack
+    (its BF16 input activation and incoming gradient), gives Y, dX and dW
+    close to the FP32 products of those inputs, as close as the quantization
+    noise of its operands allows: for relative operand noise r_a, r_b a
+    product's relative error is about sqrt(r_a^2 + r_b^2) (measured: 0.56 to
+    1.02 times it on every linear of the full stack), and 1.3 times it is
+    allowed.  A wrong, zero or uncorrelated gradient has a relative error
+    near 1 and fails;
+  * the stack-level errors against the unquantized FP32 stack are finite
+    (they grow with depth: each layer is homogeneous of degree 2 in its
+    input, with no normalisation, so relative perturbations roughly double
+    per layer; the BF16-only column shows the same growth)."""
 import math
 
 import pytest
@@ -19,12 +30,16 @@ pytestmark = pytest.mark.gpu
 def _check(res):
     assert res["oracle_rows_checked"] > 0
     assert res["oracle_mismatches"] == 0
-    rows = res["rel_err_vs_fp32"]
-    for r in rows:
+    for r in res["rel_err_vs_fp32"]:
         for k in ("act", "dx", "dw_gate_up", "dw_down"):
             assert math.isfinite(r[k]), (r, k)
-            assert r[k] < 2.0, (r, k)
-    assert rows[0]["act"] < 0.3
+    assert res["rel_err_vs_fp32"][0]["act"] < 0.3
+    assert len(res["local"]) == 2 * res["layers"]
+    for r in res["local"]:
+        for k in ("y", "dx", "dw"):
+            err, noise = r[f"{k}_local"], r[f"{k}_noise"]
+            assert 0.0 < noise < 0.3, (r, k)
+            assert err <= 1.3 * noise + 1e-3, (r, k)
 
 
 def test_swiglu_stack_small(gpu_lib):
