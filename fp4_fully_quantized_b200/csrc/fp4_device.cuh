@@ -130,6 +130,20 @@ __device__ __forceinline__ uint32_t e2m1x8_rn(const float* v) {
   return out;
 }
 
+// Byte permute: result byte k is byte sel_k of the 8 bytes {b, a} (a = 0..3,
+// b = 4..7); a selector nibble with bit 3 set replicates that byte's sign bit.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // E2M1 stochastic rounding with 16-bit draws: with lo <= |v| <= hi the
 // neighbouring levels (|v| clamped to 6) and p = (|v| - lo) / (hi - lo),
 // round up iff floor(p * 2^16) + u >= 2^16.
@@ -142,32 +156,81 @@ __device__ __forceinline__ uint32_t e2m1x8_rn(const float* v) {
 // [2^23, 2^24) every float is an integer), and the floor of the min is the
 // min of the floors.  So min(...) as an integer is 2^23 + code(lo) * 2^16 +
 // floor(p * 2^16), below 2^23 + 2^19; adding the draw carries into bit 16
-// exactly when the value rounds up, and bits 16..18 are the code.  NaN
-// inputs give 6 (fminf drops NaN); they are flagged by the amax check.
-__device__ __forceinline__ uint32_t e2m1_sr16_magnitude_bits(float v, uint32_t u16) {
-  const float a = fabsf(v);
+// exactly when the value rounds up, and byte 2 of the sum is the code (its
+// bits 3..7 stay 0).  NaN inputs give 6 (min drops NaN); they are flagged by
+// the amax check.
+__device__ __forceinline__ uint32_t sr16_byte2(float a, uint32_t u16) {
   const float g1 = __fmaf_rd(a, 131072.0f, 8388608.0f);               // a*2^17 + 2^23
   const float g2 = __fmaf_rd(a, 65536.0f, 8519680.0f);                // (a+2)*2^16 + 2^23
   const float g3 = __fmaf_rd(a, 32768.0f, 8650752.0f);                // (a+8)*2^15 + 2^23
-  const float m = fminf(fminf(g1, g2), fminf(g3, 8847360.0f));       // 7*2^16 + 2^23
-  return __float_as_uint(m) + u16;                                   // code in bits 16..18
+  const float m = fminf(fmin3(g1, g2, g3), 8847360.0f);              // 7*2^16 + 2^23
+  return __float_as_uint(m) + u16;
 }
 
-// Eight values -> eight stochastically rounded codes, element j in bits
-// 4j..4j+3 (sign kept, also for results of 0), with the 16-bit draws of one
-// Philox block: element j uses the low (j even) or high (j odd) half of
-// word j / 2.
+// Codes of 4 elements, one per byte (byte k = element k), from their sr16_byte2
+// results.
+__device__ __forceinline__ uint32_t gather_byte2(uint32_t t0, uint32_t t1, uint32_t t2, uint32_t t3) {
+  return prmt(prmt(t0, t1, 0x0062u), prmt(t2, t3, 0x0062u), 0x5410u);
+}
+
+// Eight 4-bit codes (element k in byte k of lo / hi, magnitude in bits 0..2,
+// sign in bit 3) packed into one word, element k in bits 4k..4k+3.
+__device__ __forceinline__ uint32_t pack_nibbles(uint32_t lo, uint32_t hi) {
+  lo |= lo >> 4;                                  // bytes 0 and 2 now hold two codes each
+  hi |= hi >> 4;
+  return prmt(lo, hi, 0x6420u);
+}
+
+// Magnitudes a[8] = |RN(x * inv)| of eight elements with sign bytes `sgn_lo`
+// (elements 0..3) and `sgn_hi` (4..7), byte k 0xFF for a negative element and
+// 0 otherwise: stochastically rounded E2M1 codes, element k in bits 4k..4k+3,
+// with the 16-bit draws of one Philox block (element k: the low (k even) or
+// high (k odd) half of word k / 2).
+__device__ __forceinline__ uint32_t e2m1x8_sr_mag(const float* a, uint32_t sgn_lo, uint32_t sgn_hi,
+                                                  const U4& w) {
+  const uint32_t t0 = sr16_byte2(a[0], w.x & 0xFFFFu), t1 = sr16_byte2(a[1], w.x >> 16);
+  const uint32_t t2 = sr16_byte2(a[2], w.y & 0xFFFFu), t3 = sr16_byte2(a[3], w.y >> 16);
+  const uint32_t t4 = sr16_byte2(a[4], w.z & 0xFFFFu), t5 = sr16_byte2(a[5], w.z >> 16);
+  const uint32_t t6 = sr16_byte2(a[6], w.w & 0xFFFFu), t7 = sr16_byte2(a[7], w.w >> 16);
+  const uint32_t lo = gather_byte2(t0, t1, t2, t3) | (sgn_lo & 0x08080808u);
+  const uint32_t hi = gather_byte2(t4, t5, t6, t7) | (sgn_hi & 0x08080808u);
+  return pack_nibbles(lo, hi);
+}
+
+// Sign bytes of four BF16 values held as two pairs (element 2j in the low
+// half of word j): byte k is 0xFF when element k is negative.
+__device__ __forceinline__ uint32_t bf16_sign_bytes(uint32_t w0, uint32_t w1) {
+  return prmt(w0, w1, 0xFDB9u);
+}
+
+// Sign bytes of four floats.
+__device__ __forceinline__ uint32_t f32_sign_bytes(float v0, float v1, float v2, float v3) {
+  return prmt(prmt(__float_as_uint(v0), __float_as_uint(v1), 0x00FBu),
+              prmt(__float_as_uint(v2), __float_as_uint(v3), 0x00FBu), 0x5410u);
+}
+
+// Eight signed values v[8] (already multiplied by the block's inverse scale):
+// stochastically rounded codes as e2m1x8_sr_mag.
 __device__ __forceinline__ uint32_t e2m1x8_sr(const float* v, const U4& w) {
-  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-  uint32_t out = 0;
+  float a[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const uint32_t u16 = (j & 1) ? (ws[j >> 1] >> 16) : (ws[j >> 1] & 0xFFFFu);
-    const uint32_t t = e2m1_sr16_magnitude_bits(v[j], u16);
-    const uint32_t nib = ((t >> 16) & 7u) | ((__float_as_uint(v[j]) >> 28) & 8u);
-    out |= nib << (4 * j);
-  }
-  return out;
+  for (int j = 0; j < 8; ++j) a[j] = fabsf(v[j]);
+  return e2m1x8_sr_mag(a, f32_sign_bytes(v[0], v[1], v[2], v[3]),
+                       f32_sign_bytes(v[4], v[5], v[6], v[7]), w);
+}
+
+// RN(y / 6) for the block-scale step, as Markstein's correction of a product
+// by the rounded reciprocal (P. Markstein, IBM J. Res. Dev. 34(1), 1990):
+// q0 = RN(y * RN(1/6)), e = y - 6 q0 (exact by FMA), q1 = RN(q0 + e * RN(1/6)).
+// Checked on the CPU for every non-negative binary32 y against the exactly
+// rounded quotient: equal for all y >= 2^-125; below that both quotients are
+// under 2^-127, far under half of E4M3's smallest step (2^-10), so the E4M3
+// scale chosen from them is the same for every y.
+__device__ __forceinline__ float div6_for_scale(float y) {
+  const float r = 0.16666667163372040f;              // RN(1/6) = 0x3E2AAAAB
+  const float q0 = __fmul_rn(y, r);
+  const float e = __fmaf_rn(-6.0f, q0, y);
+  return __fmaf_rn(e, r, q0);
 }
 
 // ---------------------------------------------------------------------------

@@ -339,7 +339,7 @@ fp4_gemm_sfst_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 bmax = fmaxf(bmax, fabsf(o[e]));
               }
               amax = fmaxf(amax, bmax);
-              const uint32_t sf = fp4dev::e4m3_rn_sat(__fdiv_rn(__fmul_rn(bmax, q_senc), 6.0f));
+              const uint32_t sf = fp4dev::e4m3_rn_sat(fp4dev::div6_for_scale(__fmul_rn(bmax, q_senc)));
               const float inv = (sf == 0u || sf == 127u)
                                     ? 0.0f : fminf(__fdiv_rn(q_senc, fp4dev::e4m3_value(sf)), FLT_MAX);
 #pragma unroll

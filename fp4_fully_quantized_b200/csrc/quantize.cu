@@ -277,7 +277,7 @@ quant_rows_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t col
       uint32_t sf;
       float inv;
       if constexpr (NV) {
-        const float t = __fdiv_rn(__fmul_rn(bmax, s_enc), 6.0f);
+        const float t = div6_for_scale(__fmul_rn(bmax, s_enc));
         sf = e4m3_rn_sat(t);                  // 0 .. 126
         inv = inv_tab[sf];
       } else {
@@ -294,7 +294,16 @@ quant_rows_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t col
       } else {
         // one Philox block: the 16-bit draws of these 8 elements
         const uint64_t i0 = (uint64_t)r * (uint64_t)cols + (uint64_t)(c * 8);
-        packed = e2m1x8_sr(v, philox_keyed(i0 >> 3, sr_stream, K));
+        const U4 w = philox_keyed(i0 >> 3, sr_stream, K);
+        if constexpr (RHT_N > 0) {
+          packed = e2m1x8_sr(v, w);
+        } else {
+          float a[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) a[i] = fabsf(v[i]);
+          packed = e2m1x8_sr_mag(a, bf16_sign_bytes(raw[q].x, raw[q].y),
+                                 bf16_sign_bytes(raw[q].z, raw[q].w), w);
+        }
       }
       if (c < cpr) {
         *reinterpret_cast<uint32_t*>(codes + r * (cols >> 1) + c * 4) = packed;
@@ -407,7 +416,7 @@ quant_cols_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t col
         uint32_t sf;
         float inv;
         if constexpr (NV) {
-          const float tt = __fdiv_rn(__fmul_rn(bmax, s_enc), 6.0f);
+          const float tt = div6_for_scale(__fmul_rn(bmax, s_enc));
           sf = e4m3_rn_sat(tt);
           inv = (sf == 0) ? 0.0f : fminf(__fdiv_rn(s_enc, e4m3_value(sf)), FLT_MAX);
         } else {
@@ -514,7 +523,7 @@ quant_2d_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols,
 #pragma unroll
       for (int o = 8; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xFFFFFFFFu, bm, o));
       if (rr == 0) {
-        const float tt = __fdiv_rn(__fmul_rn(bm, s_enc), 6.0f);
+        const float tt = div6_for_scale(__fmul_rn(bm, s_enc));
         const uint32_t sf = e4m3_rn_sat(tt);
         tsf[q] = sf;
         tinv[q] = (sf == 0) ? 0.0f : fminf(__fdiv_rn(s_enc, e4m3_value(sf)), FLT_MAX);
@@ -591,7 +600,7 @@ template <bool NV>
 __device__ __forceinline__ void block_scale(float bmax, float s_enc, const float* inv_tab,
                                             uint32_t& sf, float& inv) {
   if constexpr (NV) {
-    const float t = __fdiv_rn(__fmul_rn(bmax, s_enc), 6.0f);
+    const float t = div6_for_scale(__fmul_rn(bmax, s_enc));
     sf = e4m3_rn_sat(t);                  // 0 .. 126 (satfinite)
     inv = inv_tab[sf];                    // RN(s_enc / value(sf)), 0 for sf = 0
   } else {
@@ -602,11 +611,14 @@ __device__ __forceinline__ void block_scale(float bmax, float s_enc, const float
   }
 }
 
-template <int BS>
-constexpr int dual_ctas_per_sm() { return BS == 16 ? kDualCtasPerSm : 2; }
+// Resident CTAs per SM: three for the round-to-nearest NVFP4 forms (at most
+// 80 registers a thread), two where stochastic rounding or 32-value blocks
+// need more registers than that without spilling.
+template <int BS, bool SR_R, bool SR_C>
+constexpr int dual_ctas_per_sm() { return (BS == 16 && !SR_R && !SR_C) ? kDualCtasPerSm : 2; }
 
 template <int BS, int RHT_R, int RHT_C, bool SR_R, bool SR_C>
-__global__ void __launch_bounds__(kDualThreads, dual_ctas_per_sm<BS>())
+__global__ void __launch_bounds__(kDualThreads, (dual_ctas_per_sm<BS, SR_R, SR_C>()))
 quant_dual_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
                   uint32_t mask_r, uint32_t mask_c, const __grid_constant__ PhiloxKeys K,
                   uint32_t stream_r,
@@ -678,37 +690,58 @@ quant_dual_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t col
     const int64_t m0 = (tile_id / tiles_k) * kDualTM, k0 = (tile_id % tiles_k) * kDualTK;
 
     // ---------------- row phase (blocks along x's rows) -----------------
+    {
+      const int cc = lane * 8;
+      const int64_t c = k0 + cc;
+      const bool col_ok = c < cols;
+      const int64_t sb = c / BS;
+      // tensor-core scale layout, split into the tile's row-block part (r >> 7
+      // is the same for the tile's 64 rows) and this lane's block part
+      const int64_t mma_tile = (m0 >> 7) * (S_r4 >> 2) * 512 + (sb >> 2) * 512 + (sb & 3);
+      uint8_t* cptr = codes_r + (m0 + warp) * (cols >> 1) + (c >> 1);
+      const int64_t cstep = 8 * (cols >> 1);
 #pragma unroll 2
-    for (int i = 0; i < 8; ++i) {
-      const int rr = i * 8 + warp, cc = lane * 8;
-      const int64_t r = m0 + rr, c = k0 + cc;
-      const bool active = (r < rows) && (c < cols);
-      float v[8];
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(&tile[buf][rr][cc]), v);
-      if constexpr (RHT_R > 0) rht_chunk<RHT_R>(v, mask_r, lane % (RHT_R / 8));
-      float bmax = 0.0f;
+      for (int i = 0; i < 8; ++i, cptr += cstep) {
+        const int rr = i * 8 + warp;
+        const int64_t r = m0 + rr;
+        const uint4 raw = *reinterpret_cast<const uint4*>(&tile[buf][rr][cc]);
+        float v[8];
+        bf16x8_to_f32(raw, v);
+        if constexpr (RHT_R > 0) rht_chunk<RHT_R>(v, mask_r, lane % (RHT_R / 8));
+        float bmax = 0.0f;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) bmax = fmaxf(bmax, fabsf(v[q]));
+        for (int q = 0; q < 8; ++q) bmax = fmaxf(bmax, fabsf(v[q]));
 #pragma unroll
-      for (int lx = 1; lx < TPB; lx <<= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xFFFFFFFFu, bmax, lx));
-      uint32_t sf;
-      float inv;
-      block_scale<NV>(bmax, se_r, inv_tab[0], sf, inv);
+        for (int lx = 1; lx < TPB; lx <<= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xFFFFFFFFu, bmax, lx));
+        uint32_t sf;
+        float inv;
+        block_scale<NV>(bmax, se_r, inv_tab[0], sf, inv);
+        uint32_t packed;
+        if constexpr (!SR_R) {
 #pragma unroll
-      for (int q = 0; q < 8; ++q) v[q] = __fmul_rn(v[q], inv);
-      uint32_t packed;
-      if constexpr (!SR_R) {
-        packed = e2m1x8_rn(v);
-      } else {
-        const uint64_t i0 = (uint64_t)r * (uint64_t)cols + (uint64_t)c;      // a multiple of 8
-        packed = e2m1x8_sr(v, philox_keyed(i0 >> 3, stream_r, K));
-      }
-      if (active) {
-        *reinterpret_cast<uint32_t*>(codes_r + r * (cols >> 1) + (c >> 1)) = packed;
-        if ((lane % TPB) == 0) {
-          const int64_t sb = c / BS;
-          if (scales_r != nullptr) scales_r[r * S_r + sb] = (uint8_t)sf;
-          if (mma_r != nullptr) mma_r[mma_sf_offset(r, sb, S_r4)] = (uint8_t)sf;
+          for (int q = 0; q < 8; ++q) v[q] = __fmul_rn(v[q], inv);
+          packed = e2m1x8_rn(v);
+        } else {
+          // one Philox block: the 16-bit draws of these 8 elements
+          const uint64_t i0 = (uint64_t)r * (uint64_t)cols + (uint64_t)c;    // a multiple of 8
+          const U4 w = philox_keyed(i0 >> 3, stream_r, K);
+          if constexpr (RHT_R > 0) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) v[q] = __fmul_rn(v[q], inv);
+            packed = e2m1x8_sr(v, w);
+          } else {
+            float a[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) a[q] = __fmul_rn(fabsf(v[q]), inv);
+            packed = e2m1x8_sr_mag(a, bf16_sign_bytes(raw.x, raw.y), bf16_sign_bytes(raw.z, raw.w), w);
+          }
+        }
+        if (col_ok && r < rows) {
+          *reinterpret_cast<uint32_t*>(cptr) = packed;
+          if ((lane % TPB) == 0) {
+            if (scales_r != nullptr) scales_r[r * S_r + sb] = (uint8_t)sf;
+            if (mma_r != nullptr) mma_r[mma_tile + (rr & 31) * 16 + (((int)(m0 & 127) + rr) >> 5) * 4] = (uint8_t)sf;
+          }
         }
       }
     }
@@ -742,6 +775,18 @@ quant_dual_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t col
 #pragma unroll
           for (int q = 0; q < BS; ++q)
             raw[q] = *reinterpret_cast<const uint32_t*>(&tile[buf][tr0 + q][2 * p]);
+          // sign bytes of both columns, 4 rows per word (stochastic rounding
+          // without rotation takes them from the BF16 pairs directly)
+          uint32_t sgn[2][BS / 4];
+          if constexpr (SR_C && RHT_C == 0) {
+#pragma unroll
+            for (int g = 0; g < BS / 4; ++g) {
+              const uint32_t P = prmt(raw[4 * g], raw[4 * g + 1], 0xFDB9u);
+              const uint32_t Q = prmt(raw[4 * g + 2], raw[4 * g + 3], 0xFDB9u);
+              sgn[0][g] = prmt(P, Q, 0x6420u);
+              sgn[1][g] = prmt(P, Q, 0x7531u);
+            }
+          }
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             float v[BS];
@@ -773,9 +818,9 @@ quant_dual_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t col
             float inv;
             block_scale<NV>(bmax, se_c, inv_tab[1], sf, inv);
             sfw[e] |= sf << (8 * b);
-#pragma unroll
-            for (int q = 0; q < BS; ++q) v[q] = __fmul_rn(v[q], inv);
             if constexpr (!SR_C) {
+#pragma unroll
+              for (int q = 0; q < BS; ++q) v[q] = __fmul_rn(v[q], inv);
 #pragma unroll
               for (int w = 0; w < BS / 8; ++w) cw[e][b * (BS / 8) + w] = e2m1x8_rn(&v[8 * w]);
             } else {
@@ -783,8 +828,19 @@ quant_dual_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t col
               // a multiple of 8 at q = 0
               const uint64_t i0 = (uint64_t)(kc + e) * (uint64_t)rows + (uint64_t)mrow0;
 #pragma unroll
-              for (int w = 0; w < BS / 8; ++w)
-                cw[e][b * (BS / 8) + w] = e2m1x8_sr(&v[8 * w], philox_keyed((i0 >> 3) + w, stream_c, K));
+              for (int w = 0; w < BS / 8; ++w) {
+                const U4 d = philox_keyed((i0 >> 3) + w, stream_c, K);
+                if constexpr (RHT_C > 0) {
+#pragma unroll
+                  for (int q = 0; q < 8; ++q) v[8 * w + q] = __fmul_rn(v[8 * w + q], inv);
+                  cw[e][b * (BS / 8) + w] = e2m1x8_sr(&v[8 * w], d);
+                } else {
+                  float a[8];
+#pragma unroll
+                  for (int q = 0; q < 8; ++q) a[q] = __fmul_rn(fabsf(v[8 * w + q]), inv);
+                  cw[e][b * (BS / 8) + w] = e2m1x8_sr_mag(a, sgn[e][2 * w], sgn[e][2 * w + 1], d);
+                }
+              }
             }
           }
         }
@@ -929,7 +985,7 @@ static cudaError_t dual_variant(const DualQuantArgs& a, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDualSmem);
   if (e != cudaSuccess) return e;
   const int64_t ntiles = ((a.rows + kDualTM - 1) / kDualTM) * ((a.cols + kDualTK - 1) / kDualTK);
-  const int grid = grid_for(ntiles, 1, dual_ctas_per_sm<BS>());
+  const int grid = grid_for(ntiles, 1, dual_ctas_per_sm<BS, SRR, SRC>());
   kern<<<grid, kDualThreads, kDualSmem, s>>>(
       static_cast<const __nv_bfloat16*>(a.x), a.rows, a.cols, a.ld, a.mask_r, a.mask_c,
       philox_keys(a.sr_seed), a.stream_r, a.stream_c, a.amax_src_r, a.amax_src_c, a.amax_out_r,
