@@ -65,6 +65,22 @@ struct StParams {
   uint32_t* status;
 };
 
+// Tile order: groups of kGroupM row blocks are walked column block by column
+// block (row block fastest), so the tiles the persistent CTAs work on at one
+// time share few A row blocks and few B column blocks, and both stay in L2
+// while every CTA that needs them streams them (a row-major walk over all
+// column blocks streams the whole of B once per wave of tiles).
+constexpr int kGroupM = 16;
+
+__device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, int& mb, int& nb) {
+  const int per_group = kGroupM * tiles_n;
+  const int g = tile / per_group, r = tile - g * per_group;
+  const int m0 = g * kGroupM;
+  const int gm = min(kGroupM, tiles_m - m0);
+  nb = r / gm;
+  mb = m0 + (r - nb * gm);
+}
+
 // Waits with one lane and broadcasts the result to the warp.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           uint32_t* status, uint32_t where, int lane) {
@@ -130,7 +146,8 @@ fp4_gemm_sfst_kernel(const __grid_constant__ CUtensorMap tmap_a,
       uint32_t it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int mb = tile / tiles_n, nb = tile % tiles_n;
+        int mb, nb;
+        tile_coords(tile, tiles_m, tiles_n, mb, nb);
         const bool b_hi = (nb * 2 + 1) * 128 < p.N;
         for (int kb = 0; kb < k_blocks; ++kb, ++it) {
           const int s = it % STAGES;
@@ -269,7 +286,8 @@ fp4_gemm_sfst_kernel(const __grid_constant__ CUtensorMap tmap_a,
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tile_iter) {
       if (!warp_wait(acc_full, tile_iter & 1u, abort_flag, p.status, 0x3700 + warp, lane)) break;
       tc_fence_after();
-      const int mb = tile / tiles_n, nb = tile % tiles_n;
+      int mb, nb;
+      tile_coords(tile, tiles_m, tiles_n, mb, nb);
       const int64_t row = (int64_t)mb * BM + quad * 32 + lane;
       const int c_begin = half * (BN / 2);
       const int ncols = min(BN / 2, p.N - nb * BN - c_begin);

@@ -39,13 +39,16 @@
  *   - Matrices are row-major.  Packed FP4 codes: two per byte, element 2j in
  *     the low nibble of byte j.  A code is sign (bit 3), exponent (bits 2-1),
  *     mantissa (bit 0).  Pointers must be 16-byte aligned.
- *   - Stochastic-rounding draws are counter-based: element i (row-major
- *     index in the quantized operand's own logical layout) uses word i mod 4
- *     of Philox4x32-10 with key (seed lo, seed hi) and counter
- *     (i/4 lo, i/4 hi, stream, 0), so results do not depend on the launch
- *     configuration.  The Hadamard sign vector d (d_j = -1 iff bit 31 of
- *     draw j of stream 0x48414441 under the RHT seed) is shared by every
- *     block of both operands of a GEMM.
+ *   - Stochastic rounding is counter-based, 16 random bits per element:
+ *     element i (row-major index in the quantized operand's own logical
+ *     layout) takes the low (i even) or high (i odd) half of 32-bit draw
+ *     j = i/2, draw j being word j mod 4 of Philox4x32-10 with key
+ *     (seed lo, seed hi) and counter (j/4 lo, j/4 hi, stream, 0); with p the
+ *     value's fraction of the gap between its two neighbouring E2M1 levels,
+ *     it rounds up iff floor(p * 2^16) + u >= 2^16.  Results do not depend on
+ *     the launch configuration.  The Hadamard sign vector d (d_j = -1 iff
+ *     bit 31 of 32-bit draw j of stream 0x48414441 under the RHT seed) is
+ *     shared by every block of both operands of a GEMM.
  */
 #ifndef FP4FQT_FP4_H
 #define FP4FQT_FP4_H

@@ -142,6 +142,34 @@ def test_gemm_llama_fprop_sampled_rows(gpu_lib, nk):
     assert rel_fro(got, ref) <= TOL
 
 
+@pytest.mark.parametrize("mnk", [(4096, 4096, 16384), (1024, 768, 16384)])
+def test_gemm_long_k_sampled_rows(gpu_lib, mnk):
+    """A weight-gradient-like product (long contraction, FP32 output, 3.46
+    and 0.21 waves of tiles on the persistent grid): sampled rows against the
+    float64 oracle over the full contraction, and the same bits on a second
+    call."""
+    F = gpu_lib
+    M, N, K = mnk
+    a = S.normal((M, K), 1e-3, seed=21)
+    b = S.sparse_outliers(N, K, seed=22)
+    qa, qb = O.nvfp4_quantize_1d(S.as_f32(a)), O.nvfp4_quantize_1d(S.as_f32(b))
+    ta, tb = upload_qtensor(F, qa, M, K, 0, 0), upload_qtensor(F, qb, N, K, 0, 0)
+    out = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    ws = F.Workspace(M, N, K)
+    F.fp4_gemm(ta, tb, out, ws=ws)
+    again = torch.full_like(out, float("nan"))
+    F.fp4_gemm(ta, tb, again, ws=ws)
+    torch.cuda.synchronize()
+    assert ws.status() == 0
+    assert torch.equal(out, again)
+    rows = np.sort(np.random.default_rng(6).choice(M, 32, replace=False))
+    bh = O.dequantize(qb["codes"], qb["scales"])
+    ah = O.dequantize(qa["codes"][rows], qa["scales"][rows])
+    ref = O.gemm(ah, bh, s_dec_a=qa["s_dec"], s_dec_b=qb["s_dec"])
+    got = out[torch.from_numpy(rows).cuda()].cpu().numpy()
+    assert rel_fro(got, ref) <= TOL
+
+
 @pytest.mark.parametrize("mnk", SHAPES)
 def test_gemm_mxfp4_small_shapes(gpu_lib, mnk):
     _small(gpu_lib, 1, mnk)
