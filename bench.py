@@ -642,7 +642,8 @@ def run_sweep(args, device):
     return lines
 
 
-def run_swiglu(device, layers=8, hidden=2048, ffn=8192, tokens=16384, seed=0, check_rows=8):
+def run_swiglu(device, layers=8, hidden=2048, ffn=8192, tokens=16384, seed=0, check_rows=8,
+               chained=False):
     """Chained SwiGLU MLP stack through the library's linear layer: NVFP4 fprop
     through all layers (RTN, 16x16 weight tiles), then dgrad / wgrad back with
     stochastically rounded gradients.  Every linear is fqt_linear_fwd /
@@ -689,26 +690,79 @@ def run_swiglu(device, layers=8, hidden=2048, ffn=8192, tokens=16384, seed=0, ch
         h = torch.empty((M, H), dtype=torch.bfloat16, device=device)
         F.fqt_linear_fwd(cfg, a, w_d[l], h, sv_d[l], ws)
         acts.append(h)
-    d, dxs, dwg, dwd, dys, das = dy_top, [None] * L, [None] * L, [None] * L, {}, [None] * L
-    for l in reversed(range(L)):
-        dys[(l, "d")] = d
-        da = torch.empty((M, Fd), dtype=torch.bfloat16, device=device)
-        das[l] = da
-        dwd[l] = torch.empty((H, Fd), dtype=torch.float32, device=device)
-        F.fqt_linear_bwd(cfg, d, sv_d[l], da, dwd[l], ws)
-        g, u = gus[l][:, :Fd], gus[l][:, Fd:]
-        daf = da.float()
-        dgu = torch.cat([daf * u * dsilu(g), daf * silu(g)], dim=1).to(torch.bfloat16).contiguous()
-        dys[(l, "gu")] = dgu
-        dx = torch.empty((M, H), dtype=torch.bfloat16, device=device)
-        dwg[l] = torch.empty((2 * Fd, H), dtype=torch.float32, device=device)
-        F.fqt_linear_bwd(cfg, dgu, sv_gu[l], dx, dwg[l], ws)
-        dxs[l] = dx
-        d = dx
+    fwd_end = torch.cuda.Event(enable_timing=True)
+    fwd_end.record()
+
+    def backward(chain_amax=None):
+        """The backward pass.  With chain_amax (one supplied amax per block
+        boundary, from an earlier pass: delayed scaling), block l's gate_up
+        dgrad encodes block l-1's down-projection dY operand (row-wise, SR) in
+        its epilogue and also stores it as BF16; that down layer then only
+        quantizes the transposed operand, in one pass with the same supplied
+        amax.  Returns the gradients, the dY tensors each linear consumed,
+        and each block boundary's measured |dX| max."""
+        d, dxs, dwg, dwd, dys, das = dy_top, [None] * L, [None] * L, [None] * L, {}, [None] * L
+        cam = [torch.zeros(1, dtype=torch.float32, device=device) for _ in range(L)]
+        for l in reversed(range(L)):
+            dys[(l, "d")] = d
+            da = torch.empty((M, Fd), dtype=torch.bfloat16, device=device)
+            das[l] = da
+            dwd[l] = torch.empty((H, Fd), dtype=torch.float32, device=device)
+            if chain_amax is not None and l < L - 1:
+                sv = sv_d[l]          # sv.dyq was encoded by block l + 1's dgrad epilogue
+                F.fp4_quantize(d, None, sv.dyq_t, round_t=F.SR, sr_seed=seed, sr_stream_t=2,
+                               amax_in_t=chain_amax[l], ws=ws)
+                F.fp4_gemm(sv.dyq, sv.wq_t, da, ws=ws)
+                F.fp4_gemm(sv.dyq_t, sv.xq_t, dwd[l], ws=ws)
+            else:
+                F.fqt_linear_bwd(cfg, d, sv_d[l], da, dwd[l], ws)
+            g, u = gus[l][:, :Fd], gus[l][:, Fd:]
+            daf = da.float()
+            dgu = torch.cat([daf * u * dsilu(g), daf * silu(g)], dim=1).to(torch.bfloat16).contiguous()
+            dys[(l, "gu")] = dgu
+            dx = torch.empty((M, H), dtype=torch.bfloat16, device=device)
+            dwg[l] = torch.empty((2 * Fd, H), dtype=torch.float32, device=device)
+            if chain_amax is not None and l > 0:
+                sv = sv_gu[l]
+                F.fp4_quantize(dgu, sv.dyq, sv.dyq_t, round=F.SR, round_t=F.SR, sr_seed=seed,
+                               sr_stream=1, sr_stream_t=2, ws=ws)
+                F.fp4_gemm_quant_ex(sv.dyq, sv.wq_t, sv_d[l - 1].dyq, chain_amax[l - 1], round=F.SR,
+                                    sr_seed=seed, sr_stream=1, c_bf16=dx, c_amax=cam[l - 1], ws=ws)
+                F.fp4_gemm(sv.dyq_t, sv.xq_t, dwg[l], ws=ws)
+            else:
+                F.fqt_linear_bwd(cfg, dgu, sv_gu[l], dx, dwg[l], ws)
+                if l > 0:
+                    cam[l - 1].copy_(dx.float().abs().max().reshape(1))
+            dxs[l] = dx
+            d = dx
+        return dxs, dwg, dwd, dys, das, cam
+
+    dxs, dwg, dwd, dys, das, cam = backward()
     t1.record()
     torch.cuda.synchronize()
     assert ws.status() == 0, f"device status {ws.status()}"
     ms = t0.elapsed_time(t1)
+    ms_bwd = fwd_end.elapsed_time(t1)
+    chain = None
+    if chained:
+        # delayed scaling: this pass encodes with the amax the previous pass measured
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record()
+        dxs, dwg, dwd, dys, das, cam2 = backward(chain_amax=cam)
+        c1.record()
+        torch.cuda.synchronize()
+        assert ws.status() == 0, f"device status {ws.status()}"
+        n_dx = (L - 1) * M * H            # gradient elements crossing a block boundary
+        chain = {"ms_bwd_chained": round(c0.elapsed_time(c1), 3), "ms_bwd_unchained": round(ms_bwd, 3),
+                 "boundaries": L - 1,
+                 # per element of such a gradient: the unchained path writes BF16 (2 B),
+                 # reads it for the amax (2 B) and for the fused row + transposed encode
+                 # (2 B); chained, the epilogue writes BF16 and the row-wise codes, and
+                 # one transposed-only pass reads the BF16 once
+                 "hbm_bytes_removed": n_dx * 2,
+                 "bf16_reads_removed": n_dx * 2 * 2 // 2,
+                 "amax_supplied_vs_measured": [[float(a.item()), float(b.item())]
+                                               for a, b in zip(cam[:L - 1], cam2[:L - 1])]}
     # gradient norm against the SR quantization noise of each layer's dY
     # (the two quantities the "FP4 All the Way" page relates)
     sums = torch.zeros(2, dtype=torch.float64, device=device)
@@ -811,6 +865,8 @@ def run_swiglu(device, layers=8, hidden=2048, ffn=8192, tokens=16384, seed=0, ch
     for l in sorted(chk):
         for sv, xin, dyin in ((sv_gu[l], hin[2 * l], dys[(l, "gu")]), (sv_d[l], hin[2 * l + 1], dys[(l, "d")])):
             for q, src, rnd, stream in ((sv.xq, xin, "rtn", 0), (sv.dyq, dyin, "sr", 1)):
+                if chained and q is sv.dyq and sv is sv_d[l] and l < L - 1:
+                    continue      # encoded from the FP32 product in the epilogue, not from dyin
                 rows_ = np.sort(rng.choice(M, check_rows, replace=False))
                 amax = float(q.amax.item())
                 C_ = src.shape[1]
@@ -826,7 +882,8 @@ def run_swiglu(device, layers=8, hidden=2048, ffn=8192, tokens=16384, seed=0, ch
     return {"case": "swiglu", "layers": L, "hidden": H, "ffn": Fd, "tokens": M,
             "ms_quantized_fwd_bwd": round(ms, 3),
             "tflops_gemm_equiv": round(L * 6 * M * (2 * Fd * H + H * Fd) / (ms * 1e-3) / 1e12, 1),
-            "rel_err_vs_fp32": per_layer, "local": local, "oracle_rows_checked": checked,
+            "rel_err_vs_fp32": per_layer, "local": local, "chained": chain,
+            "oracle_rows_checked": checked,
             "oracle_mismatches": mism}
 
 
@@ -913,6 +970,9 @@ def main():
                     help="data parallel: sum each layer's dW over the ranks (NCCL) inside the step")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--chained", action="store_true",
+                    help="--case swiglu: also run the backward with each block's dgrad epilogue "
+                         "encoding the next block's dY operand (delayed amax)")
     ap.add_argument("--no-sweep", action="store_true",
                     help="skip the compact quantizer sweep (config 3 at 2^28) after the step")
     ap.add_argument("--e2e-steps", type=int, default=2)
@@ -934,7 +994,7 @@ def main():
             for line in run_sweep(args, dev):
                 print(json.dumps(line), flush=True)
         elif args.case == "swiglu":
-            print(json.dumps(run_swiglu(dev, seed=args.seed)), flush=True)
+            print(json.dumps(run_swiglu(dev, seed=args.seed, chained=args.chained)), flush=True)
         else:
             print(json.dumps(run_case(args, dev)), flush=True)
         return

@@ -34,7 +34,7 @@ EXPORTS = ("fp4_qtensor_sizes", "fp4_qparams_default", "fp4_workspace_bytes", "f
            "fp4_gemm", "fqt_linear_cfg_default", "fqt_linear_fwd", "fqt_linear_bwd",
            "fp4_read_device_status", "fp4_clear_device_status", "fp4_status_str",
            "fp4_abi_version", "fp4_kernel_launches", "fp4_gemm_noalloc", "fp4_mma_rate",
-           "fp4_quant_noise", "fp4_gemm_quant")
+           "fp4_quant_noise", "fp4_gemm_quant", "fp4_gemm_quant_ex")
 
 
 class Fp4Error(RuntimeError):
@@ -115,6 +115,10 @@ def load() -> C.CDLL:
     L.fp4_gemm_quant.restype = i32
     L.fp4_gemm_quant.argtypes = [C.POINTER(QTensorC), C.POINTER(QTensorC), C.c_float, vp,
                                  C.POINTER(QTensorC), vp, vp, sz, vp]
+    L.fp4_gemm_quant_ex.restype = i32
+    L.fp4_gemm_quant_ex.argtypes = [C.POINTER(QTensorC), C.POINTER(QTensorC), C.c_float, vp, i32,
+                                    C.c_uint64, C.c_uint32, C.POINTER(QTensorC), vp, i64, vp, vp,
+                                    sz, vp]
     L.fp4_quant_noise.restype = i32
     L.fp4_quant_noise.argtypes = [vp, i64, i64, i64, C.POINTER(QTensorC), vp, vp, sz, vp]
     L.fp4_gemm_noalloc.restype = i32
@@ -272,6 +276,23 @@ def fp4_gemm_quant(a: QTensor, b: QTensor, out: QTensor, amax_in: torch.Tensor, 
     code = load().fp4_gemm_quant(C.byref(a.c), C.byref(b.c), float(alpha), _ptr(amax_in),
                                  C.byref(out.c), _ptr(c_amax), ws.ptr, ws.nbytes, _stream(stream))
     _check(code, "fp4_gemm_quant")
+
+
+def fp4_gemm_quant_ex(a: QTensor, b: QTensor, out: QTensor, amax_in: torch.Tensor,
+                      round: int = RTN, sr_seed: int = 0, sr_stream: int = 0,
+                      c_bf16: torch.Tensor | None = None, alpha: float = 1.0,
+                      c_amax: torch.Tensor | None = None, ws: Workspace | None = None, stream=None):
+    """fp4_gemm_quant with RTN or SR encoding and an optional BF16 copy of the
+    FP32 result (c_bf16, [M, >= N] BF16 CUDA tensor)."""
+    if ws is None:
+        ws = Workspace(a.rows, b.rows, a.cols, device=amax_in.device)
+    if c_bf16 is not None:
+        assert c_bf16.dtype == torch.bfloat16 and c_bf16.is_cuda and c_bf16.stride(1) == 1
+    code = load().fp4_gemm_quant_ex(C.byref(a.c), C.byref(b.c), float(alpha), _ptr(amax_in),
+                                    int(round), int(sr_seed), int(sr_stream), C.byref(out.c),
+                                    _ptr(c_bf16), c_bf16.stride(0) if c_bf16 is not None else 0,
+                                    _ptr(c_amax), ws.ptr, ws.nbytes, _stream(stream))
+    _check(code, "fp4_gemm_quant_ex")
 
 
 def fp4_quant_noise(x: torch.Tensor, q: QTensor, sums: torch.Tensor, ws: Workspace | None = None,

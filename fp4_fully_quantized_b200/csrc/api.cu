@@ -320,9 +320,10 @@ fp4_status fp4_gemm(const fp4_qtensor* a, const fp4_qtensor* b, float alpha, voi
 }
 
 
-fp4_status fp4_gemm_quant(const fp4_qtensor* a, const fp4_qtensor* b, float alpha,
-                          const float* out_amax_in, fp4_qtensor* out, float* c_amax, void* ws,
-                          size_t ws_bytes, void* stream) {
+static fp4_status gemm_quant_impl(const fp4_qtensor* a, const fp4_qtensor* b, float alpha,
+                                  const float* out_amax_in, int32_t round, uint64_t sr_seed,
+                                  uint32_t sr_stream, fp4_qtensor* out, void* c_bf16, int64_t ldc,
+                                  float* c_amax, void* ws, size_t ws_bytes, void* stream) {
   if (a == nullptr || b == nullptr || out == nullptr || out_amax_in == nullptr) return FP4_ERR_NULL;
   if (a->codes == nullptr || b->codes == nullptr || a->scales_mma == nullptr ||
       b->scales_mma == nullptr || a->s_dec == nullptr || b->s_dec == nullptr)
@@ -332,6 +333,7 @@ fp4_status fp4_gemm_quant(const fp4_qtensor* a, const fp4_qtensor* b, float alph
     return FP4_ERR_NULL;
   if (a->fmt != b->fmt || (a->fmt != FP4_NVFP4 && a->fmt != FP4_MXFP4)) return FP4_ERR_FORMAT;
   if (out->fmt != FP4_NVFP4 || out->block != FP4_BLOCK_1D) return FP4_ERR_FORMAT;
+  if (round != FP4_RTN && round != FP4_SR) return FP4_ERR_FORMAT;
   const int64_t M = a->rows, N = b->rows, K = a->cols;
   if (b->cols != K || out->rows != M || out->cols != N) return FP4_ERR_SHAPE;
   if (M <= 0 || N <= 0 || K <= 0 || M % 128 || N % 128 || K % 64) return FP4_ERR_SHAPE;
@@ -342,16 +344,33 @@ fp4_status fp4_gemm_quant(const fp4_qtensor* a, const fp4_qtensor* b, float alph
       (reinterpret_cast<uintptr_t>(out->scales_mma) & 3u) ||
       (reinterpret_cast<uintptr_t>(out->scales) & 3u))
     return FP4_ERR_ALIGN;
+  if (c_bf16 != nullptr && (ldc < N || (ldc * 2) % 16 || !aligned16(c_bf16))) return FP4_ERR_ALIGN;
   if (ws == nullptr || ws_bytes < fp4_workspace_bytes(M, N, K)) return FP4_ERR_WORKSPACE;
   GemmArgs g{};
   g.a_codes = a->codes; g.a_sf = a->scales_mma; g.a_sdec = a->s_dec;
   g.b_codes = b->codes; g.b_sf = b->scales_mma; g.b_sdec = b->s_dec;
   g.M = M; g.N = N; g.K = K; g.fmt = a->fmt; g.alpha = alpha;
-  g.c = nullptr; g.ldc = N; g.out_mode = 2;
+  g.c = c_bf16; g.ldc = c_bf16 ? ldc : N; g.out_mode = 2;
   g.q_codes = out->codes; g.q_scales = out->scales; g.q_scales_mma = out->scales_mma;
   g.q_amax_in = out_amax_in; g.q_amax_out = out->amax; g.q_s_dec = out->s_dec;
+  g.q_sr = round == FP4_SR; g.q_seed = sr_seed; g.q_stream = sr_stream;
   g.c_amax = c_amax; g.status = status_ptr(ws);
   return gemm_launch(g, as_stream(stream));
+}
+
+fp4_status fp4_gemm_quant(const fp4_qtensor* a, const fp4_qtensor* b, float alpha,
+                          const float* out_amax_in, fp4_qtensor* out, float* c_amax, void* ws,
+                          size_t ws_bytes, void* stream) {
+  return gemm_quant_impl(a, b, alpha, out_amax_in, FP4_RTN, 0, 0, out, nullptr, 0, c_amax, ws,
+                         ws_bytes, stream);
+}
+
+fp4_status fp4_gemm_quant_ex(const fp4_qtensor* a, const fp4_qtensor* b, float alpha,
+                             const float* out_amax_in, int32_t round, uint64_t sr_seed,
+                             uint32_t sr_stream, fp4_qtensor* out, void* c_bf16, int64_t ldc,
+                             float* c_amax, void* ws, size_t ws_bytes, void* stream) {
+  return gemm_quant_impl(a, b, alpha, out_amax_in, round, sr_seed, sr_stream, out, c_bf16, ldc,
+                         c_amax, ws, ws_bytes, stream);
 }
 
 void fqt_linear_cfg_default(fqt_linear_cfg* cfg, int32_t fmt) {

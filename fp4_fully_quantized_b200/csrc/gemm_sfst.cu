@@ -62,6 +62,9 @@ struct StParams {
   float* c_amax;
   uint8_t* q_codes; uint8_t* q_scales; uint8_t* q_scales_mma;
   const float* q_amax_in; float* q_amax_out; float* q_s_dec;
+  int q_sr;                   // out_mode 2: stochastic rounding (else to nearest)
+  uint32_t q_stream;          // its Philox stream; keys below
+  fp4dev::PhiloxKeys q_keys;
   uint32_t* status;
 };
 
@@ -357,13 +360,38 @@ fp4_gemm_sfst_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 bmax = fmaxf(bmax, fabsf(o[e]));
               }
               amax = fmaxf(amax, bmax);
+              const int64_t cb = col + 64 * h2 + 16 * b;   // first column of the block
+              if (p.c != nullptr) {
+                // the FP32 result also leaves as BF16 (for a consumer that
+                // still needs it, e.g. the transposed quantization)
+                uint32_t pk[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  __nv_bfloat162 b2 = __floats2bfloat162_rn(o[2 * e], o[2 * e + 1]);
+                  memcpy(&pk[e], &b2, 4);
+                }
+                __nv_bfloat16* bd = static_cast<__nv_bfloat16*>(p.c) + row * p.ldc + cb;
+                if (wide_st) {
+                  st_global_v8(bd, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
+                } else {
+                  reinterpret_cast<uint4*>(bd)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                  reinterpret_cast<uint4*>(bd)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                }
+              }
               const uint32_t sf = fp4dev::e4m3_rn_sat(fp4dev::div6_for_scale(__fmul_rn(bmax, q_senc)));
               const float inv = (sf == 0u || sf == 127u)
                                     ? 0.0f : fminf(__fdiv_rn(q_senc, fp4dev::e4m3_value(sf)), FLT_MAX);
 #pragma unroll
               for (int e = 0; e < 16; ++e) o[e] = __fmul_rn(o[e], inv);
-              cw[2 * b] = fp4dev::e2m1x8_rn(o);
-              cw[2 * b + 1] = fp4dev::e2m1x8_rn(o + 8);
+              if (p.q_sr) {
+                // draws of elements row * N + cb .. + 15: two Philox blocks
+                const uint64_t i0 = (uint64_t)row * (uint64_t)p.N + (uint64_t)cb;
+                cw[2 * b] = fp4dev::e2m1x8_sr(o, fp4dev::philox_keyed(i0 >> 3, p.q_stream, p.q_keys));
+                cw[2 * b + 1] = fp4dev::e2m1x8_sr(o + 8, fp4dev::philox_keyed((i0 >> 3) + 1, p.q_stream, p.q_keys));
+              } else {
+                cw[2 * b] = fp4dev::e2m1x8_rn(o);
+                cw[2 * b + 1] = fp4dev::e2m1x8_rn(o + 8);
+              }
               sfw |= sf << (8 * b);
             }
             const int64_t c0 = col + 64 * h2;              // first column of these 4 blocks
@@ -474,6 +502,7 @@ fp4_status gemm_launch(const GemmArgs& g, cudaStream_t s) {
   p.alpha = g.alpha; p.c = g.c; p.ldc = g.ldc; p.out_mode = g.out_mode;
   p.q_codes = g.q_codes; p.q_scales = g.q_scales; p.q_scales_mma = g.q_scales_mma;
   p.q_amax_in = g.q_amax_in; p.q_amax_out = g.q_amax_out; p.q_s_dec = g.q_s_dec;
+  p.q_sr = g.q_sr; p.q_stream = g.q_stream; p.q_keys = fp4dev::philox_keys(g.q_seed);
   p.c_amax = g.c_amax; p.status = g.status;
   const int tiles = (int)(g.M / BM) * (int)((g.N + BN - 1) / BN);
   const int grid = tiles < sm_count() ? tiles : sm_count();

@@ -91,6 +91,7 @@ struct GemmArgs {
   // out_mode 2: the quantized output [M, N] and the supplied tensor amax
   uint8_t* q_codes; uint8_t* q_scales; uint8_t* q_scales_mma;
   const float* q_amax_in; float* q_amax_out; float* q_s_dec;
+  int q_sr; uint64_t q_seed; uint32_t q_stream;   // out_mode 2 rounding
   uint32_t* status;
 };
 fp4_status gemm_launch(const GemmArgs& g, cudaStream_t s);

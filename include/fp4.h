@@ -198,6 +198,23 @@ fp4_status fp4_gemm_quant(const fp4_qtensor* a, const fp4_qtensor* b, float alph
                           const float* out_amax_in, fp4_qtensor* out, float* c_amax, void* ws,
                           size_t ws_bytes, void* stream);
 
+/* fp4_gemm_quant with a choice of rounding and an optional BF16 copy:
+ *   - round FP4_RTN or FP4_SR.  Stochastic rounding uses the library's
+ *     16-bit draws of (sr_seed, sr_stream) with element index m * N + n of
+ *     the [M, N] output, exactly as fp4_quantize rounds a row-wise output
+ *     ("FP4 All the Way", Key points: stochastic rounding for gradients);
+ *   - c_bf16 (nullable): the same FP32 results also stored as BF16,
+ *     [M, ldc] with ldc >= N and ldc * 2 a multiple of 16 bytes, for a
+ *     consumer that still needs them -- the transposed quantization of a
+ *     gradient (blocks down the columns), which one thread per output row
+ *     cannot form in the epilogue.
+ * Everything else as fp4_gemm_quant (which is this call with FP4_RTN and no
+ * BF16 copy). */
+fp4_status fp4_gemm_quant_ex(const fp4_qtensor* a, const fp4_qtensor* b, float alpha,
+                             const float* out_amax_in, int32_t round, uint64_t sr_seed,
+                             uint32_t sr_stream, fp4_qtensor* out, void* c_bf16, int64_t ldc,
+                             float* c_amax, void* ws, size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------------- */
 /* Linear layer  Y = X W^T  with X [M, K], W [N, K], dY [M, N]:            */
 /*   fprop  Y  = X . W^T      (contract K)                                 */

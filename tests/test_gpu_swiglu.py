@@ -51,3 +51,32 @@ def test_swiglu_stack_full_config(gpu_lib):
     res = bench.run_swiglu(torch.device("cuda", 0))
     print(res)
     _check(res)
+
+
+def _check_chained(res):
+    _check(res)
+    c = res["chained"]
+    assert c is not None and c["boundaries"] == res["layers"] - 1
+    pairs = c["amax_supplied_vs_measured"]
+    for supplied, measured in pairs:
+        assert supplied > 0 and measured > 0
+    # the boundary below the top block sees identical inputs in both passes:
+    # the amax the earlier pass measured on the BF16 gradient and the one
+    # this pass measures on the FP32 product differ by BF16 rounding only
+    supplied, measured = pairs[-1]
+    assert abs(supplied - measured) <= 2 ** -8 * measured
+
+
+def test_swiglu_stack_chained_small(gpu_lib):
+    """The backward with each block's gate_up dgrad encoding the previous
+    block's down-projection dY operand in its epilogue (SR, delayed amax)
+    keeps every linear within its operands' quantization noise of the FP32
+    products of its own inputs."""
+    _check_chained(bench.run_swiglu(torch.device("cuda", 0), layers=3, hidden=256, ffn=512,
+                                    tokens=1024, chained=True))
+
+
+def test_swiglu_stack_chained_full_config(gpu_lib):
+    res = bench.run_swiglu(torch.device("cuda", 0), chained=True)
+    print(res["chained"])
+    _check_chained(res)
