@@ -95,6 +95,10 @@ def lib():
                                          u8p, u8p]
         L.orc_dequantize.restype = None
         L.orc_dequantize.argtypes = [u8p, u8p, i64, i64, i32, i32, i32, f64p]
+        L.orc_quest_threshold.restype = C.c_float
+        L.orc_quest_threshold.argtypes = [f32p]
+        L.orc_quest_alpha.restype = C.c_float
+        L.orc_quest_alpha.argtypes = []
         L.orc_set_threads.restype = i32
         L.orc_set_threads.argtypes = [i32]
         L.orc_num_threads.restype = i32
@@ -252,14 +256,30 @@ def nvfp4_quantize_2d(x, amax_in=None) -> dict:
             "s_dec": np.float32(d.value)}
 
 
+def quest_threshold(block) -> float:
+    """The QuEST-style clipping threshold RN(alpha * RMS) of one 32-value
+    block (binary32 tree sum of squares)."""
+    b = _f32(block).reshape(-1)
+    assert b.size == 32
+    return float(lib().orc_quest_threshold(b))
+
+
+def quest_alpha() -> float:
+    return float(lib().orc_quest_alpha())
+
+
+_MODES = {"rtn": 0, "sr": 1, "quest": 2}
+
+
 def mxfp4_quantize(x, round_mode: str = "rtn", rht_n: int = 0, rht_seed: int = 0,
                    sr_seed: int = 0, sr_stream: int = 0, row_offset: int = 0) -> dict:
-    """MXFP4 1x32 quantization of the rows of x (float32 [R, C])."""
+    """MXFP4 1x32 quantization of the rows of x (float32 [R, C]); round_mode
+    "rtn", "sr", or "quest" (RMS-based clipping scale, then round to nearest)."""
     x = _f32(x)
     R, Cc = x.shape
     codes = np.zeros((R, Cc // 2), np.uint8)
     scales = np.zeros((R, Cc // 32), np.uint8)
-    rc = lib().orc_mxfp4_quantize(x, R, Cc, row_offset, 0 if round_mode == "rtn" else 1,
+    rc = lib().orc_mxfp4_quantize(x, R, Cc, row_offset, _MODES[round_mode],
                                   rht_n, rht_seed, sr_seed, sr_stream, codes, scales)
     if rc != 0:
         raise ValueError(f"oracle mxfp4_quantize rejected shape {x.shape} rht_n={rht_n}")

@@ -466,6 +466,42 @@ int orc_nvfp4_quantize_2d(const float* x, int64_t R, int64_t C, const float* ama
 /* then E2M1 rounding (values in (6, 8) saturate); b = 0 gives scale byte 0 */
 /* and zero codes.                                                          */
 /* ------------------------------------------------------------------------ */
+/* ------------------------------------------------------------------------ */
+/* QuEST-style MXFP4 forward block scale.  [Quartet] Approach and Measured  */
+/* effects (ablations): the forward pass uses a QuEST-style quantizer --     */
+/* Hadamard rotation, then clipping -- instead of plain round-to-nearest.   */
+/* The pages give no clipping rule.  reading: the block's scale comes from  */
+/* its root-mean-square instead of its maximum: T = RN(alpha * RMS), with   */
+/* alpha the clipping multiple that minimises the mean squared error of     */
+/* E2M1 round-to-nearest for a unit Gaussian (values beyond alpha clip to   */
+/* the top level), and the OCP MX power-of-two rule applied to T in place   */
+/* of the block max: e = floor(log2 T) - 2, clamped to [-127, 127]; values  */
+/* whose scaled magnitude exceeds 6 saturate (the clipping).  T = 0 gives   */
+/* scale byte 0 and zero codes, as a zero block does.                       */
+/* The mean square of the 32 values is summed in binary32 in a fixed tree:  */
+/* four groups of 8 consecutive values, each ((y0^2 + y1^2) + (y2^2 +       */
+/* y3^2)) + ((y4^2 + y5^2) + (y6^2 + y7^2)), then (g0 + g1) + (g2 + g3);    */
+/* RMS = RN(sqrt(RN(sum / 32))).                                            */
+/* ------------------------------------------------------------------------ */
+#define QUEST_ALPHA 2.9224751f
+
+float orc_quest_threshold(const float* y) {
+  float g[4];
+  for (int k = 0; k < 4; ++k) {
+    const float* v = y + 8 * k;
+    float a = v[0] * v[0] + v[1] * v[1];
+    float b = v[2] * v[2] + v[3] * v[3];
+    float c = v[4] * v[4] + v[5] * v[5];
+    float d = v[6] * v[6] + v[7] * v[7];
+    g[k] = (a + b) + (c + d);
+  }
+  float sum = (g[0] + g[1]) + (g[2] + g[3]);
+  float rms = sqrtf(sum / 32.0f);
+  return QUEST_ALPHA * rms;
+}
+
+float orc_quest_alpha(void) { return QUEST_ALPHA; }
+
 static void mxfp4_rows_worker(void* p, int64_t r0, int64_t r1) {
   q1d_ctx* q = (q1d_ctx*)p;
   const int64_t C = q->C, nb = C / 32;
@@ -477,7 +513,9 @@ static void mxfp4_rows_worker(void* p, int64_t r0, int64_t r1) {
         float a = fabsf(row[b * 32 + j]);
         if (a > bmax) bmax = a;
       }
-      int e = (bmax == 0.0f) ? -127 : orc_floor_log2(bmax) - 2;
+      /* round_mode 2 (QuEST): the clipping threshold replaces the block max */
+      float top = (q->round_mode == 2) ? orc_quest_threshold(row + b * 32) : bmax;
+      int e = (top == 0.0f) ? -127 : orc_floor_log2(top) - 2;
       if (e < -127) e = -127;
       if (e > 127) e = 127;
       q->scales[r * nb + b] = (uint8_t)(e + 127);
@@ -486,7 +524,7 @@ static void mxfp4_rows_worker(void* p, int64_t r0, int64_t r1) {
         int64_t c = b * 32 + j;
         float v = row[c] * mul;
         uint8_t code;
-        if (q->round_mode == 0) {
+        if (q->round_mode != 1) {
           code = orc_e2m1_rtn(v);
         } else {
           uint64_t idx = (uint64_t)(q->row_offset + r) * (uint64_t)C + (uint64_t)c;

@@ -23,7 +23,7 @@ from conftest import ROOT
 
 PINS = [os.path.join(ROOT, "tests", f) for f in
         ("test_oracle_formats.py", "test_oracle_quant.py", "test_oracle_rht.py",
-         "test_oracle_sr_philox.py")]
+         "test_oracle_sr_philox.py", "test_oracle_quest.py")]
 
 # (name, text in fp4_oracle.c, replacement, which occurrence to replace)
 MUTANTS = [
@@ -79,7 +79,7 @@ MUTANTS = [
     ("Hadamard butterfly sign", "v[j + h] = a - b;", "v[j + h] = b - a;", 0),
     ("Hadamard random signs dropped", "for (int j = 0; j < n; ++j) v[j] = v[j] * d[j];",
      "for (int j = 0; j < n; ++j) v[j] = v[j];", 0),
-    ("MXFP4 exponent offset", "orc_floor_log2(bmax) - 2;", "orc_floor_log2(bmax) - 1;", 0),
+    ("MXFP4 exponent offset", "orc_floor_log2(top) - 2;", "orc_floor_log2(top) - 1;", 0),
     ("MXFP4 scale byte bias", "(uint8_t)(e + 127);", "(uint8_t)(e + 128);", 0),
     ("E8M0 decode bias", "return ldexp(1.0, (int)b - 127);", "return ldexp(1.0, (int)b - 126);", 0),
     ("amax of signed values", "float a = fabsf(x[i]);", "float a = x[i];", 0),
@@ -102,6 +102,15 @@ MUTANTS = [
      "if (A == 0.0f) { *s_enc = 1.0f; *s_dec = 0.0f; return; }", 0),
     ("reciprocal of a zero scale not zero", "float inv = (sf == 0) ? 0.0f : q->s_enc / sfv;",
      "float inv = (sf == 0) ? 1.0f : q->s_enc / sfv;", 0),
+    ("QuEST alpha of 3", "#define QUEST_ALPHA 2.9224751f", "#define QUEST_ALPHA 3.0f", 0),
+    ("QuEST mean over 31", "float rms = sqrtf(sum / 32.0f);", "float rms = sqrtf(sum / 31.0f);", 0),
+    ("QuEST without the square root", "float rms = sqrtf(sum / 32.0f);", "float rms = sum / 32.0f;", 0),
+    ("QuEST last group dropped", "float sum = (g[0] + g[1]) + (g[2] + g[3]);",
+     "float sum = (g[0] + g[1]) + g[2];", 0),
+    ("QuEST scale from the block max", "float top = (q->round_mode == 2) ? orc_quest_threshold(row + b * 32) : bmax;",
+     "float top = bmax;", 0),
+    ("QuEST rounds stochastically", "        if (q->round_mode != 1) {\n          code = orc_e2m1_rtn(v);",
+     "        if (q->round_mode == 0) {\n          code = orc_e2m1_rtn(v);", 0),
 ]
 
 
