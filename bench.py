@@ -180,7 +180,9 @@ def qparams_for(cfg, which):
                     rht_n=rn if m & 1 else 0, rht_n_t=rn if m & 4 else 0, rht_seed=cfg.seed,
                     sr_seed=cfg.seed, sr_stream=0, sr_stream_t=3)
     if which == "w":
-        return dict(fmt=cfg.fmt, block=cfg.w_block, round=cfg.round_fwd, round_t=cfg.round_fwd,
+        # W^T feeds dgrad: the QuEST-style forward scale does not apply there
+        return dict(fmt=cfg.fmt, block=cfg.w_block, round=cfg.round_fwd,
+                    round_t=0 if cfg.round_fwd == 2 else cfg.round_fwd,
                     rht_n=rn if m & 1 else 0, rht_n_t=rn if m & 2 else 0, rht_seed=cfg.seed)
     return dict(fmt=cfg.fmt, round=cfg.round_bwd, round_t=cfg.round_bwd,
                 rht_n=rn if m & 2 else 0, rht_n_t=rn if m & 4 else 0, rht_seed=cfg.seed,
@@ -388,6 +390,8 @@ def run_ours(args, rank, world, device):
     cfg = F.linear_cfg(fmt, out_dtype=F.OUT_BF16, seed=args.seed)
     if args.wgrad_rht and fmt == F.NVFP4:
         cfg.rht_mask = F.RHT_WGRAD
+    if args.quest and fmt == F.MXFP4:
+        cfg.round_fwd = F.QUEST           # Quartet: QuEST-style forward quantizer
     layers, cache = make_layers(F, cfg, device, args.seed + rank)
     ws = F.Workspace(device=device)
     dp = DwAllReduce(world) if args.dp_allreduce else None
@@ -887,6 +891,68 @@ def run_swiglu(device, layers=8, hidden=2048, ffn=8192, tokens=16384, seed=0, ch
             "oracle_mismatches": mism}
 
 
+def run_formats(device, seed=0, rows_checked=128, M=M_TOKENS):
+    """Config 4: MXFP4 against NVFP4 on the same seeded Llama-7B tensors.
+
+    Per distinct layer shape and operand (X, W, dY), the relative
+    quantization noise ||deq(q(x)) - x|| / ||x|| of the row-wise operand,
+    rounded to nearest without rotation in both formats (NVFP4 weights in
+    16x16 tiles, as its layer stores them; the layer's stochastically rounded
+    NVFP4 dY is listed beside as dY_sr), from fp4_quant_noise; and the relative
+    Frobenius error of the layer's three products, each format in its own
+    layer configuration (NVFP4 without Hadamard, MXFP4 with the 32-point
+    transform on every operand), on `rows_checked` sampled output rows
+    against the unquantized float64 product of the BF16 inputs.  The "FP4"
+    page (Components, NVFP4) says NVFP4 has the lower quantization error."""
+    import fp4_fully_quantized_b200 as F
+    import fqt_synth as S
+    F.load()
+    ws = F.Workspace(device=device)
+    sums = torch.zeros(2, dtype=torch.float64, device=device)
+    rng = np.random.default_rng(seed + 11)
+    out = {"case": "formats", "tokens": M, "rows_checked": rows_checked, "shapes": []}
+    for name, N, K in [("qkvo", 4096, 4096), ("gate_up", 11008, 4096), ("down", 4096, 11008)]:
+        d = S.llama_linear(N, K, M=M, seed=seed)
+        X, W, dY = d["X"].to(device), d["W"].to(device), d["dY"].to(device)
+        row = {"layer": name, "N": N, "K": K, "noise": {}, "gemm_err": {}}
+        for fmt_name, fmt in (("nvfp4", F.NVFP4), ("mxfp4", F.MXFP4)):
+            nz = {}
+            ops = [("X", X, F.BLOCK_1D, F.RTN), ("W", W, F.BLOCK_2D, F.RTN),
+                   ("dY", dY, F.BLOCK_1D, F.RTN)]
+            if fmt == F.NVFP4:
+                ops.append(("dY_sr", dY, F.BLOCK_1D, F.SR))
+            for opn, t, blk, rnd in ops:
+                if fmt == F.MXFP4:
+                    blk = F.BLOCK_1D
+                q = F.QTensor.empty(t.shape[0], t.shape[1], fmt, blk, device=device, logical_scales=False)
+                F.fp4_quantize(t, q, fmt=fmt, block=blk, round=rnd, sr_seed=seed, sr_stream=1, ws=ws)
+                F.fp4_quant_noise(t, q, sums, ws)
+                sx, sn = sums.tolist()
+                nz[opn] = round((sn / sx) ** 0.5, 5)
+                del q
+            row["noise"][fmt_name] = nz
+            cfg = F.linear_cfg(fmt, out_dtype=F.OUT_F32, seed=seed)
+            sv = F.Saved.empty(M, N, K, cfg, device=device, logical_scales=False)
+            y = torch.empty((M, N), dtype=torch.float32, device=device)
+            dx = torch.empty((M, K), dtype=torch.float32, device=device)
+            dw = torch.empty((N, K), dtype=torch.float32, device=device)
+            F.fqt_linear_fwd(cfg, X, W, y, sv, ws)
+            F.fqt_linear_bwd(cfg, dY, sv, dx, dw, ws)
+            torch.cuda.synchronize()
+            assert ws.status() == 0
+            r = torch.from_numpy(np.sort(rng.choice(M, rows_checked, replace=False))).to(device)
+            c = torch.from_numpy(np.sort(rng.choice(N, rows_checked, replace=False))).to(device)
+            Xd, Wd, dYd = X.double(), W.double(), dY.double()
+            refs = {"Y": (Xd[r] @ Wd.t(), y[r]), "dX": (dYd[r] @ Wd, dx[r]),
+                    "dW": (dYd[:, c].t() @ Xd, dw[c])}
+            row["gemm_err"][fmt_name] = {k: round(float((g.double() - ref).norm() / ref.norm()), 5)
+                                         for k, (ref, g) in refs.items()}
+            del sv, y, dx, dw
+        out["shapes"].append(row)
+        del X, W, dY
+    return out
+
+
 def run_case(args, device):
     """A single kernel family on one small problem (for profiler captures):
     --case gemm: NVFP4 fprop-style GEMM [m, k] x [n, k]^T, BF16 out;
@@ -948,7 +1014,7 @@ def run_case(args, device):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--case", choices=["gemm", "gemm_quant", "gemm_then_quant", "quant", "quant_sr",
-                                       "sweep", "swiglu"], default=None,
+                                       "sweep", "swiglu", "formats"], default=None,
                     help="time one kernel family on one problem (profiling), or the "
                          "quantizer sweep over 2^n elements")
     ap.add_argument("--rounds", default=None,
@@ -966,6 +1032,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--fmt", choices=["nvfp4", "mxfp4"], default="nvfp4")
     ap.add_argument("--wgrad-rht", action="store_true")
+    ap.add_argument("--quest", action="store_true",
+                    help="--fmt mxfp4: QuEST-style forward quantizer (RMS-based clipping scale)")
     ap.add_argument("--dp-allreduce", action="store_true",
                     help="data parallel: sum each layer's dW over the ranks (NCCL) inside the step")
     ap.add_argument("--seed", type=int, default=0)
@@ -993,6 +1061,8 @@ def main():
         if args.case == "sweep":
             for line in run_sweep(args, dev):
                 print(json.dumps(line), flush=True)
+        elif args.case == "formats":
+            print(json.dumps(run_formats(dev, seed=args.seed)), flush=True)
         elif args.case == "swiglu":
             print(json.dumps(run_swiglu(dev, seed=args.seed, chained=args.chained)), flush=True)
         else:

@@ -20,7 +20,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libfp4fqt.so")
 
 NVFP4, MXFP4 = 0, 1
-RTN, SR = 0, 1
+RTN, SR, QUEST = 0, 1, 2
 BLOCK_1D, BLOCK_2D = 0, 1
 OUT_BF16, OUT_F32 = 0, 1
 RHT_FPROP, RHT_DGRAD, RHT_WGRAD = 1, 2, 4

@@ -132,8 +132,13 @@ static fp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64
   if (p->fmt != FP4_NVFP4 && p->fmt != FP4_MXFP4) return FP4_ERR_FORMAT;
   if (p->block != FP4_BLOCK_1D && p->block != FP4_BLOCK_2D) return FP4_ERR_FORMAT;
   if (p->block == FP4_BLOCK_2D && p->fmt != FP4_NVFP4) return FP4_ERR_FORMAT;
-  if ((p->round != FP4_RTN && p->round != FP4_SR) || (p->round_t != FP4_RTN && p->round_t != FP4_SR))
+  if ((p->round != FP4_RTN && p->round != FP4_SR && p->round != FP4_QUEST) ||
+      (p->round_t != FP4_RTN && p->round_t != FP4_SR && p->round_t != FP4_QUEST))
     return FP4_ERR_FORMAT;
+  // the QuEST-style scale is defined for MXFP4 row-wise (forward) outputs
+  if (p->round == FP4_QUEST && (p->fmt != FP4_MXFP4 || p->block != FP4_BLOCK_1D))
+    return FP4_ERR_UNSUPPORTED;
+  if (out_t != nullptr && p->round_t == FP4_QUEST) return FP4_ERR_UNSUPPORTED;
   for (int n : {p->rht_n, p->rht_n_t})
     if (n != 0 && n != 16 && n != 32) return FP4_ERR_FORMAT;
   const int bs = block_size(p->fmt);
@@ -232,6 +237,7 @@ static fp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64
     a.x = x; a.rows = rows; a.cols = cols; a.ld = ld;
     a.fmt = p->fmt; a.rht_r = p->rht_n; a.rht_c = p->rht_n_t;
     a.sr_r = p->round == FP4_SR; a.sr_c = p->round_t == FP4_SR;
+    a.quest_r = p->round == FP4_QUEST;
     a.mask_r = mask; a.mask_c = mask_t;
     a.sr_seed = p->sr_seed; a.stream_r = p->sr_stream; a.stream_c = p->sr_stream_t;
     a.amax_src_r = src_row; a.amax_src_c = src_col;
@@ -394,6 +400,8 @@ void fqt_linear_cfg_default(fqt_linear_cfg* cfg, int32_t fmt) {
 static fp4_status check_cfg(const fqt_linear_cfg* cfg) {
   if (cfg == nullptr) return FP4_ERR_NULL;
   if (cfg->fmt != FP4_NVFP4 && cfg->fmt != FP4_MXFP4) return FP4_ERR_FORMAT;
+  if (cfg->round_bwd == FP4_QUEST || cfg->round_x_t == FP4_QUEST) return FP4_ERR_UNSUPPORTED;
+  if (cfg->round_fwd == FP4_QUEST && cfg->fmt != FP4_MXFP4) return FP4_ERR_UNSUPPORTED;
   if (cfg->rht_mask & ~7) return FP4_ERR_FORMAT;
   if (cfg->rht_mask && cfg->rht_n != 16 && cfg->rht_n != 32) return FP4_ERR_FORMAT;
   if (cfg->w_block == FP4_BLOCK_2D) {
@@ -433,7 +441,7 @@ fp4_status fqt_linear_fwd(const fqt_linear_cfg* cfg, int64_t M, int64_t N, int64
   pw.fmt = cfg->fmt;
   pw.block = cfg->w_block;
   pw.round = cfg->round_fwd;
-  pw.round_t = cfg->round_fwd;
+  pw.round_t = cfg->round_fwd == FP4_QUEST ? FP4_RTN : cfg->round_fwd;   // W^T feeds dgrad
   pw.rht_n = (cfg->rht_mask & FQT_RHT_FPROP) ? rn : 0;
   pw.rht_n_t = (cfg->rht_mask & FQT_RHT_DGRAD) ? rn : 0;
   pw.rht_seed = cfg->seed;

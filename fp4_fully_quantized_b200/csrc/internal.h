@@ -59,6 +59,7 @@ cudaError_t launch_quant_cols(const RowQuantArgs& a, cudaStream_t s);
 struct DualQuantArgs {
   const void* x; int64_t rows, cols, ld;
   int fmt, rht_r, rht_c; bool sr_r, sr_c;
+  bool quest_r;            // MXFP4 row-wise output: QuEST-style (RMS-based) block scale
   uint32_t mask_r, mask_c;
   uint64_t sr_seed; uint32_t stream_r, stream_c;
   const float* amax_src_r; const float* amax_src_c;   // NVFP4 (ignored for MXFP4)

@@ -52,6 +52,26 @@ __device__ __forceinline__ void rht_chunk(float* v, uint32_t mask, int q) {
   }
 }
 
+// QuEST-style clipping threshold of an MXFP4 32-block held by four adjacent
+// lanes (8 consecutive values each, lane % 4 = group): T = RN(alpha * RMS)
+// with the mean square summed in binary32 as ((y0^2 + y1^2) + (y2^2 + y3^2))
+// + ((y4^2 + y5^2) + (y6^2 + y7^2)) per lane, then (g0 + g1) + (g2 + g3) over
+// the lanes (two butterfly stages; both orders of each add give the same
+// bits); alpha = 2.9224751 minimises the E2M1 rounding MSE of a unit
+// Gaussian ("Quartet", Approach: QuEST-style forward quantization).
+constexpr float kQuestAlpha = 2.9224751f;
+
+__device__ __forceinline__ float quest_threshold(const float* v) {
+  const float a = __fadd_rn(__fmul_rn(v[0], v[0]), __fmul_rn(v[1], v[1]));
+  const float b = __fadd_rn(__fmul_rn(v[2], v[2]), __fmul_rn(v[3], v[3]));
+  const float c = __fadd_rn(__fmul_rn(v[4], v[4]), __fmul_rn(v[5], v[5]));
+  const float d = __fadd_rn(__fmul_rn(v[6], v[6]), __fmul_rn(v[7], v[7]));
+  float g = __fadd_rn(__fadd_rn(a, b), __fadd_rn(c, d));
+  g = __fadd_rn(g, __shfl_xor_sync(0xFFFFFFFFu, g, 1));
+  g = __fadd_rn(g, __shfl_xor_sync(0xFFFFFFFFu, g, 2));
+  return __fmul_rn(kQuestAlpha, __fsqrt_rn(__fmul_rn(g, 0.03125f)));
+}
+
 __device__ __forceinline__ void block_amax_atomic(float m, float* amax) {
   __shared__ float red[kThreads / 32];
 #pragma unroll
@@ -217,7 +237,7 @@ amax_cols_rht_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t 
 // ---------------------------------------------------------------------------
 constexpr int kRowChunks = 4;
 
-template <int BS, int RHT_N, bool SR>
+template <int BS, int RHT_N, bool SR, bool QUEST = false>
 __global__ void __launch_bounds__(kThreads)
 quant_rows_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
                   uint32_t rht_mask, const __grid_constant__ PhiloxKeys K, uint32_t sr_stream,
@@ -281,7 +301,9 @@ quant_rows_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t col
         sf = e4m3_rn_sat(t);                  // 0 .. 126
         inv = inv_tab[sf];
       } else {
-        int e = (bmax == 0.0f) ? -127 : floor_log2_f32(bmax) - 2;
+        // QuEST: the clipping threshold takes the block max's place
+        const float top = QUEST ? quest_threshold(v) : bmax;
+        int e = (top == 0.0f) ? -127 : floor_log2_f32(top) - 2;
         e = max(-127, min(127, e));
         sf = (uint32_t)(e + 127);
         inv = exp2_neg_exact(e);
@@ -617,7 +639,7 @@ __device__ __forceinline__ void block_scale(float bmax, float s_enc, const float
 template <int BS, bool SR_R, bool SR_C>
 constexpr int dual_ctas_per_sm() { return (BS == 16 && !SR_R && !SR_C) ? kDualCtasPerSm : 2; }
 
-template <int BS, int RHT_R, int RHT_C, bool SR_R, bool SR_C>
+template <int BS, int RHT_R, int RHT_C, bool SR_R, bool SR_C, bool QUEST_R = false>
 __global__ void __launch_bounds__(kDualThreads, (dual_ctas_per_sm<BS, SR_R, SR_C>()))
 quant_dual_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
                   uint32_t mask_r, uint32_t mask_c, const __grid_constant__ PhiloxKeys K,
@@ -715,7 +737,12 @@ quant_dual_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t col
         for (int lx = 1; lx < TPB; lx <<= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xFFFFFFFFu, bmax, lx));
         uint32_t sf;
         float inv;
-        block_scale<NV>(bmax, se_r, inv_tab[0], sf, inv);
+        if constexpr (QUEST_R) {
+          // QuEST (MXFP4): the clipping threshold takes the block max's place
+          block_scale<NV>(quest_threshold(v), se_r, inv_tab[0], sf, inv);
+        } else {
+          block_scale<NV>(bmax, se_r, inv_tab[0], sf, inv);
+        }
         uint32_t packed;
         if constexpr (!SR_R) {
 #pragma unroll
@@ -935,9 +962,9 @@ cudaError_t launch_amax_cols(const void* x, int64_t rows, int64_t cols, int64_t 
   return cudaGetLastError();
 }
 
-template <int BS, int RHT_N, bool SR>
+template <int BS, int RHT_N, bool SR, bool QUEST = false>
 static void rows_variant(const RowQuantArgs& a, int grid, cudaStream_t s) {
-  quant_rows_kernel<BS, RHT_N, SR><<<grid, kThreads, 0, s>>>(
+  quant_rows_kernel<BS, RHT_N, SR, QUEST><<<grid, kThreads, 0, s>>>(
       static_cast<const __nv_bfloat16*>(a.x), a.rows, a.cols, a.ld, a.rht_mask, philox_keys(a.sr_seed),
       a.sr_stream, a.amax_src, a.amax_out, a.s_dec, a.codes, a.scales, a.scales_mma, a.status);
 }
@@ -966,6 +993,13 @@ static void cols_variant(const RowQuantArgs& a, int grid, cudaStream_t s) {
 cudaError_t launch_quant_rows(const RowQuantArgs& a, cudaStream_t s) {
   const int64_t segs = ((a.cols / 8) + 32 * kRowChunks - 1) / (32 * kRowChunks);
   const int grid = grid_for(a.rows * segs, kThreads / 32, 8);
+  if (a.round == FP4_QUEST) {       // MXFP4 only (checked by the caller)
+    if (a.rht_n == 32) rows_variant<32, 32, false, true>(a, grid, s);
+    else if (a.rht_n == 16) rows_variant<32, 16, false, true>(a, grid, s);
+    else rows_variant<32, 0, false, true>(a, grid, s);
+    count_launches(1);
+    return cudaGetLastError();
+  }
   FP4_DISPATCH(rows_variant, a, grid, s);
   count_launches(1);
   return cudaGetLastError();
@@ -979,9 +1013,9 @@ cudaError_t launch_quant_cols(const RowQuantArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-template <int BS, int RR, int RC, bool SRR, bool SRC>
+template <int BS, int RR, int RC, bool SRR, bool SRC, bool QR = false>
 static cudaError_t dual_variant(const DualQuantArgs& a, cudaStream_t s) {
-  auto kern = quant_dual_kernel<BS, RR, RC, SRR, SRC>;
+  auto kern = quant_dual_kernel<BS, RR, RC, SRR, SRC, QR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDualSmem);
   if (e != cudaSuccess) return e;
   const int64_t ntiles = ((a.rows + kDualTM - 1) / kDualTM) * ((a.cols + kDualTK - 1) / kDualTK);
@@ -997,6 +1031,10 @@ static cudaError_t dual_variant(const DualQuantArgs& a, cudaStream_t s) {
 
 template <int BS, int RR, int RC>
 static cudaError_t dual_rounding(const DualQuantArgs& a, cudaStream_t s) {
+  if constexpr (BS == 32) {
+    if (a.quest_r) return a.sr_c ? dual_variant<BS, RR, RC, false, true, true>(a, s)
+                                 : dual_variant<BS, RR, RC, false, false, true>(a, s);
+  }
   if (a.sr_r) return a.sr_c ? dual_variant<BS, RR, RC, true, true>(a, s)
                             : dual_variant<BS, RR, RC, true, false>(a, s);
   return a.sr_c ? dual_variant<BS, RR, RC, false, true>(a, s)

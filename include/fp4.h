@@ -80,7 +80,7 @@ typedef enum fp4_status {
 
 /* Values of the int32_t selector fields below. */
 enum { FP4_NVFP4 = 0, FP4_MXFP4 = 1 };            /* format                  */
-enum { FP4_RTN = 0, FP4_SR = 1 };                 /* rounding                */
+enum { FP4_RTN = 0, FP4_SR = 1, FP4_QUEST = 2 };  /* rounding (see below)    */
 enum { FP4_BLOCK_1D = 0, FP4_BLOCK_2D = 1 };      /* 1x16 / 1x32, or 16x16    */
 enum { FP4_OUT_BF16 = 0, FP4_OUT_F32 = 1 };       /* GEMM output type         */
 enum { FQT_RHT_FPROP = 1, FQT_RHT_DGRAD = 2, FQT_RHT_WGRAD = 4 };
@@ -133,7 +133,15 @@ void fp4_qtensor_sizes(int64_t rows, int64_t cols, int32_t fmt, int32_t block,
 typedef struct fp4_qparams {
   int32_t fmt;            /* FP4_NVFP4 or FP4_MXFP4                                  */
   int32_t block;          /* FP4_BLOCK_1D, or FP4_BLOCK_2D (NVFP4 weights, RTN only) */
-  int32_t round;          /* rounding of the row-wise output                         */
+  int32_t round;          /* rounding of the row-wise output: FP4_RTN, FP4_SR, or    */
+                          /* FP4_QUEST (MXFP4 only): the QuEST-style forward scale   */
+                          /* of "Quartet" (Approach): each 32-block's scale from     */
+                          /* T = RN(2.9224751 * RMS) by the power-of-two rule         */
+                          /* floor(log2 T) - 2 in place of the block max (values      */
+                          /* beyond the top level clip), then round to nearest; the  */
+                          /* mean square is summed in binary32 as ((y0^2 + y1^2) +   */
+                          /* (y2^2 + y3^2)) + ((y4^2 + y5^2) + (y6^2 + y7^2)) per    */
+                          /* group of 8, then (g0 + g1) + (g2 + g3)                  */
   int32_t round_t;        /* rounding of the transposed output                       */
   int32_t rht_n;          /* 0, 16 or 32: Hadamard block of the row-wise output      */
   int32_t rht_n_t;        /* 0, 16 or 32: Hadamard block of the transposed output    */
@@ -224,7 +232,8 @@ fp4_status fp4_gemm_quant_ex(const fp4_qtensor* a, const fp4_qtensor* b, float a
 typedef struct fqt_linear_cfg {
   int32_t fmt;        /* FP4_NVFP4 or FP4_MXFP4                                   */
   int32_t w_block;    /* NVFP4: FP4_BLOCK_2D (16x16 weight tiles) or FP4_BLOCK_1D  */
-  int32_t round_fwd;  /* rounding of X and W for fprop                            */
+  int32_t round_fwd;  /* rounding of X and W for fprop (FP4_QUEST: MXFP4 only;    */
+                      /* W^T for dgrad then rounds to nearest)                    */
   int32_t round_bwd;  /* rounding of dY (dgrad and wgrad operands)                */
   int32_t round_x_t;  /* rounding of X^T, the wgrad ("update pass") operand       */
   int32_t rht_mask;   /* FQT_RHT_* bits: GEMMs whose operands are rotated first    */

@@ -24,7 +24,7 @@ def _oracle_layer(X, W, dY, cfg):
     nv = cfg.fmt == 0
     T = lambda a: np.ascontiguousarray(a.T)
     rn, seed, m = cfg.rht_n, cfg.seed, cfg.rht_mask
-    r = lambda rnd: "sr" if rnd == 1 else "rtn"
+    r = lambda rnd: {0: "rtn", 1: "sr", 2: "quest"}[rnd]
 
     def q1(a, rnd, rht, stream):
         if nv:
@@ -46,7 +46,8 @@ def _oracle_layer(X, W, dY, cfg):
         wblk = (16, 16)
     else:
         ops["wq"] = q1(W, cfg.round_fwd, rn if m & 1 else 0, 0)
-        ops["wq_t"] = q1(T(W), cfg.round_fwd, rn if m & 2 else 0, 0)
+        # W^T feeds dgrad: the QuEST-style forward scale does not apply there
+        ops["wq_t"] = q1(T(W), 0 if cfg.round_fwd == 2 else cfg.round_fwd, rn if m & 2 else 0, 0)
         wblk = (1, 16)
     ops["dyq"] = q1(dY, cfg.round_bwd, rn if m & 2 else 0, 1)
     ops["dyq_t"] = q1(T(dY), cfg.round_bwd, rn if m & 4 else 0, 2)
@@ -85,12 +86,15 @@ def _compare_ops(F, sv, ops, cfg):
         assert float(t.s_dec.item()) == float(ref["s_dec"]), name
 
 
-@pytest.mark.parametrize("variant", ["nvfp4", "nvfp4_wgrad_rht", "nvfp4_1d_rht_all", "mxfp4"])
+@pytest.mark.parametrize("variant", ["nvfp4", "nvfp4_wgrad_rht", "nvfp4_1d_rht_all", "mxfp4",
+                                     "mxfp4_quest"])
 def test_tiny_linear_layer(gpu_lib, variant):
     F = gpu_lib
     d = S.tiny_linear(seed=0)
-    fmt = 1 if variant == "mxfp4" else 0
+    fmt = 1 if variant.startswith("mxfp4") else 0
     cfg = F.linear_cfg(fmt, out_dtype=F.OUT_F32)
+    if variant == "mxfp4_quest":
+        cfg.round_fwd = F.QUEST           # Quartet: QuEST-style forward, RTN backward
     if variant == "nvfp4_wgrad_rht":
         cfg.rht_mask = F.RHT_WGRAD
     if variant == "nvfp4_1d_rht_all":

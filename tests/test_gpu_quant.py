@@ -151,6 +151,37 @@ def test_mxfp4_rows_and_transposed(gpu_lib, shape, rnd, rht):
     _check_1d(qt, O.mxfp4_quantize(np.ascontiguousarray(xf.T), sr_stream=5, **kw), 1)
 
 
+@pytest.mark.parametrize("shape", [(128, 256), (64, 96), (256, 4096), (32, 64)])
+@pytest.mark.parametrize("rht", [0, 32])
+@pytest.mark.parametrize("with_t", [False, True])
+def test_mxfp4_quest_rows(gpu_lib, shape, rht, with_t):
+    """MXFP4 with the QuEST-style forward scale on the row-wise output, alone
+    (row kernel) and beside a round-to-nearest transposed output (fused
+    kernel): codes and scales bit-exact with the oracle."""
+    F = gpu_lib
+    R, Cc = shape
+    if rht and (Cc % rht or (with_t and R % rht)):
+        pytest.skip("Hadamard block must divide the blocked dimension")
+    x = S.sparse_outliers(R, Cc, seed=13)
+    q, qt = _gpu_quant(F, x, 1, round=F.QUEST, round_t=RTN, rht_n=rht, rht_n_t=rht, seed=4,
+                       col=with_t)
+    xf = S.as_f32(x)
+    _check_1d(q, O.mxfp4_quantize(xf, "quest", rht_n=rht, rht_seed=4), 1)
+    if with_t:
+        _check_1d(qt, O.mxfp4_quantize(np.ascontiguousarray(xf.T), rht_n=rht, rht_seed=4), 1)
+
+
+def test_quest_requests_outside_mxfp4_rows_are_rejected(gpu_lib):
+    F = gpu_lib
+    x = S.normal((64, 64), 1.0, seed=1).cuda()
+    with pytest.raises(F.Fp4Error) as e:
+        F.fp4_quantize(x, F.QTensor.empty(64, 64), round=F.QUEST)            # NVFP4
+    assert e.value.code == 9
+    with pytest.raises(F.Fp4Error) as e:
+        F.fp4_quantize(x, None, F.QTensor.empty(64, 64, F.MXFP4), fmt=F.MXFP4, round_t=F.QUEST)
+    assert e.value.code == 9
+
+
 @pytest.mark.parametrize("case", ["nvfp4_rtn", "nvfp4_sr", "nvfp4_2d", "mxfp4", "nvfp4_ragged"])
 def test_quant_noise_matches_oracle(gpu_lib, case):
     """fp4_quant_noise (sum x^2, sum (deq - x)^2 in double) against the
