@@ -298,13 +298,14 @@ fp4_gemm_sfst_kernel(const __grid_constant__ CUtensorMap tmap_a,
       const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)c_begin;
       if (p.out_mode == 0) {
         // drain 128 columns in two 64-column loads, packing to BF16 as they
-        // arrive (64 registers); two TMEM round trips before the release
+        // arrive (64 registers); the accumulator is released as soon as the
+        // second load has landed, before that half is packed, so the next
+        // tile's MMAs wait for two TMEM round trips and one packing only
         uint32_t pk[64];
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
+        {
           uint32_t r2[64];
-          tmem_ld32_nowait(taddr + 64 * q, r2);
-          tmem_ld32_nowait(taddr + 64 * q + 32, r2 + 32);
+          tmem_ld32_nowait(taddr, r2);
+          tmem_ld32_nowait(taddr + 32, r2 + 32);
           asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
           for (int h = 0; h < 32; ++h) {
@@ -312,12 +313,26 @@ fp4_gemm_sfst_kernel(const __grid_constant__ CUtensorMap tmap_a,
             const float a1 = __uint_as_float(r2[2 * h + 1]) * scale;
             amax = fmaxf(amax, fmaxf(fabsf(a0), fabsf(a1)));
             __nv_bfloat162 b2 = __floats2bfloat162_rn(a0, a1);
-            memcpy(&pk[32 * q + h], &b2, 4);
+            memcpy(&pk[h], &b2, 4);
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(acc_empty);
+        {
+          uint32_t r2[64];
+          tmem_ld32_nowait(taddr + 64, r2);
+          tmem_ld32_nowait(taddr + 96, r2 + 32);
+          asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(acc_empty);
+#pragma unroll
+          for (int h = 0; h < 32; ++h) {
+            const float a0 = __uint_as_float(r2[2 * h]) * scale;
+            const float a1 = __uint_as_float(r2[2 * h + 1]) * scale;
+            amax = fmaxf(amax, fmaxf(fabsf(a0), fabsf(a1)));
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(a0, a1);
+            memcpy(&pk[32 + h], &b2, 4);
+          }
+        }
         if (ncols > 0) {
           __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.c) + row * p.ldc + col;
           if (wide_st) {          // full 32-byte sectors
