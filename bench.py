@@ -191,20 +191,35 @@ def qparams_for(cfg, which):
 
 class DwAllReduce:
     """Data-parallel gradient exchange: each layer's FP32 dW [N, K] summed over
-    all ranks.  It is issued right after that layer's wgrad; NCCL runs it on
-    its own stream, after the work already queued, so it overlaps the next
+    all ranks.  It is issued right after that layer's wgrad and runs on a
+    stream of its own, after the work already queued, so it overlaps the next
     layer's kernels.  `finish` makes the launching stream wait for every
-    pending sum; every rank issues the same sums in the same order."""
+    pending sum; every rank issues the same sums in the same order.
 
-    def __init__(self, world: int):
-        self.world, self.works = world, []
+    With `F` and `comm` (an F.NcclComm) the sums go through the library's
+    fp4_allreduce_sum_f32 (NCCL on the comm stream); without them, through
+    torch.distributed (any backend: the CPU tests run it on gloo)."""
+
+    def __init__(self, world: int, F=None, comm=None):
+        self.world, self.works, self.F, self.comm = world, [], F, comm
+        self.stream = torch.cuda.Stream() if comm is not None else None
 
     def issue(self, dw: torch.Tensor):
         """Starts the sum of dw after the work queued on the current stream;
         returns its handle (None on one rank)."""
         if self.world <= 1:
             return None
-        work = torch.distributed.all_reduce(dw, async_op=True)
+        if self.comm is None:
+            work = torch.distributed.all_reduce(dw, async_op=True)
+            self.works.append(work)
+            return work
+        ready = torch.cuda.Event()
+        ready.record()
+        self.stream.wait_event(ready)
+        self.F.fp4_allreduce_sum_f32(self.comm, dw, stream=self.stream)
+        done = torch.cuda.Event()
+        done.record(self.stream)
+        work = _StreamWork(done)
         self.works.append(work)
         return work
 
@@ -212,6 +227,17 @@ class DwAllReduce:
         for w in self.works:
             w.wait()
         self.works.clear()
+
+
+class _StreamWork:
+    """A sum enqueued on the comm stream: wait() orders the current stream
+    after it (the torch work handle's meaning for NCCL)."""
+
+    def __init__(self, event):
+        self.event = event
+
+    def wait(self):
+        torch.cuda.current_stream().wait_event(self.event)
 
 
 def plan(F, layers, ws, dp=None):
@@ -394,7 +420,10 @@ def run_ours(args, rank, world, device):
         cfg.round_fwd = F.QUEST           # Quartet: QuEST-style forward quantizer
     layers, cache = make_layers(F, cfg, device, args.seed + rank)
     ws = F.Workspace(device=device)
-    dp = DwAllReduce(world) if args.dp_allreduce else None
+    dp = None
+    if args.dp_allreduce:
+        comm = F.NcclComm(rank, world) if world > 1 else None
+        dp = DwAllReduce(world, F, comm)
     calls = plan(F, layers, ws, dp)
     clk = ClockSampler(device.index).__enter__()     # sampling before the timed region
     for _ in range(args.warmup):
@@ -986,7 +1015,8 @@ def run_case(args, device):
         qbt = F.QTensor.empty(K, N, F.NVFP4, F.BLOCK_2D, device=device, logical_scales=False)
         F.fp4_quantize(x, qa, ws=ws)
         F.fp4_quantize(w, qb, qbt, block=F.BLOCK_2D, ws=ws)
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        y = torch.empty((M, N), dtype=torch.float32 if args.out == "f32" else torch.bfloat16,
+                        device=device)
         qy = F.QTensor.empty(M, N, device=device, logical_scales=False)
         y_amax = torch.ones(1, dtype=torch.float32, device=device)   # supplied (delayed) amax
         if args.case == "gemm_quant":          # result encoded to NVFP4 in the epilogue
@@ -1023,6 +1053,8 @@ def main():
                     help="--case quant: supply the tensor amax (times the fused encode alone)")
     ap.add_argument("--sweep-min", type=int, default=20)
     ap.add_argument("--sweep-max", type=int, default=30)
+    ap.add_argument("--out", choices=["bf16", "f32"], default="bf16",
+                    help="--case gemm: output type (the weight gradient is FP32)")
     ap.add_argument("--m", type=int, default=8192)
     ap.add_argument("--n", type=int, default=4096)
     ap.add_argument("--k", type=int, default=4096)

@@ -34,7 +34,7 @@ EXPORTS = ("fp4_qtensor_sizes", "fp4_qparams_default", "fp4_workspace_bytes", "f
            "fp4_gemm", "fqt_linear_cfg_default", "fqt_linear_fwd", "fqt_linear_bwd",
            "fp4_read_device_status", "fp4_clear_device_status", "fp4_status_str",
            "fp4_abi_version", "fp4_kernel_launches", "fp4_gemm_noalloc", "fp4_mma_rate",
-           "fp4_quant_noise", "fp4_gemm_quant", "fp4_gemm_quant_ex")
+           "fp4_quant_noise", "fp4_gemm_quant", "fp4_gemm_quant_ex", "fp4_allreduce_sum_f32")
 
 
 class Fp4Error(RuntimeError):
@@ -119,6 +119,8 @@ def load() -> C.CDLL:
     L.fp4_gemm_quant_ex.argtypes = [C.POINTER(QTensorC), C.POINTER(QTensorC), C.c_float, vp, i32,
                                     C.c_uint64, C.c_uint32, C.POINTER(QTensorC), vp, i64, vp, vp,
                                     sz, vp]
+    L.fp4_allreduce_sum_f32.restype = i32
+    L.fp4_allreduce_sum_f32.argtypes = [vp, vp, i64, vp]
     L.fp4_quant_noise.restype = i32
     L.fp4_quant_noise.argtypes = [vp, i64, i64, i64, C.POINTER(QTensorC), vp, vp, sz, vp]
     L.fp4_gemm_noalloc.restype = i32
@@ -304,6 +306,53 @@ def fp4_quant_noise(x: torch.Tensor, q: QTensor, sums: torch.Tensor, ws: Workspa
                                   _ptr(sums), ws.ptr if ws is not None else None,
                                   ws.nbytes if ws is not None else 0, _stream(stream))
     _check(code, "fp4_quant_noise")
+
+
+class NcclComm:
+    """An NCCL communicator for fp4_allreduce_sum_f32 (plumbing only): made
+    with the process's NCCL, its unique id passed from rank 0 to the others
+    through the torch.distributed process group `group` (any backend)."""
+
+    def __init__(self, rank: int, world: int, group=None):
+        import torch.distributed as dist
+        self._nccl = C.CDLL("libnccl.so.2", mode=os.RTLD_NOLOAD | os.RTLD_LAZY) \
+            if _nccl_loaded() else C.CDLL("libnccl.so.2")
+        uid = _NcclUniqueId()
+        if rank == 0 and self._nccl.ncclGetUniqueId(C.byref(uid)) != 0:
+            raise RuntimeError("ncclGetUniqueId failed")
+        if world > 1:
+            box = [bytes(uid.internal)]
+            dist.broadcast_object_list(box, src=0, group=group)
+            C.memmove(C.byref(uid), box[0], 128)
+        self.comm = C.c_void_p()
+        self._nccl.ncclCommInitRank.argtypes = [C.POINTER(C.c_void_p), C.c_int, _NcclUniqueId, C.c_int]
+        if self._nccl.ncclCommInitRank(C.byref(self.comm), world, uid, rank) != 0:
+            raise RuntimeError("ncclCommInitRank failed")
+
+    def destroy(self):
+        if self.comm:
+            self._nccl.ncclCommDestroy(self.comm)
+            self.comm = C.c_void_p()
+
+
+class _NcclUniqueId(C.Structure):
+    """ncclUniqueId: 128 opaque bytes, passed to ncclCommInitRank by value."""
+    _fields_ = [("internal", C.c_char * 128)]
+
+
+def _nccl_loaded() -> bool:
+    try:
+        C.CDLL("libnccl.so.2", mode=os.RTLD_NOLOAD | os.RTLD_LAZY)
+        return True
+    except OSError:
+        return False
+
+
+def fp4_allreduce_sum_f32(comm: NcclComm, buf: torch.Tensor, stream=None):
+    """buf (FP32 CUDA tensor) <- its sum over the communicator's ranks."""
+    assert buf.dtype == torch.float32 and buf.is_cuda and buf.is_contiguous()
+    _check(load().fp4_allreduce_sum_f32(comm.comm, _ptr(buf), buf.numel(), _stream(stream)),
+           "fp4_allreduce_sum_f32")
 
 
 def linear_cfg(fmt: int = NVFP4, **overrides) -> LinearCfgC:

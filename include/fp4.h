@@ -301,6 +301,19 @@ fp4_status fqt_linear_bwd(const fqt_linear_cfg* cfg, int64_t M, int64_t N, int64
 fp4_status fp4_gemm_noalloc(const fp4_qtensor* a, const fp4_qtensor* b, float alpha, void* c,
                             int64_t ldc, int32_t out_dtype, float* c_amax, void* stream);
 
+/* Data-parallel weight-gradient sum: buf[0 .. count) (FP32, device memory)
+ * is replaced by its sum over the ranks of `nccl_comm` (an ncclComm_t the
+ * caller created, passed as void*), enqueued with NCCL on `stream` after the
+ * work already queued there (typically the layer's wgrad).  The one exchange
+ * of data-parallel training of the layer: every rank quantizes its own token
+ * shard and computes its own dW ("FP4 All the Way", Summary: the 7B model
+ * trained on 256 accelerators).  Every rank must make the same calls in the
+ * same order.  The library does not link NCCL: the process's NCCL is found
+ * by its soname (libnccl.so.2) on first use; FP4_ERR_UNSUPPORTED when there
+ * is none, FP4_ERR_CUDA when NCCL reports an error.  count == 0 does
+ * nothing. */
+fp4_status fp4_allreduce_sum_f32(void* nccl_comm, float* buf, int64_t count, void* stream);
+
 /* Gradient-norm vs quantization-noise diagnostic ("FP4 All the Way" page,
  * Summary: quantized training stops being effective below a threshold set
  * by the relation between the gradient norm and the quantization noise; the

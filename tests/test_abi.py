@@ -183,3 +183,13 @@ def test_gemm_rejects_tile_counts_beyond_32_bits(lib):
     b2 = _q((1 << 15) + 256, 128)
     assert lib.fp4_gemm(C.byref(a), C.byref(b2), 1.0, c, (1 << 15) + 256, 0, None, ws, 256,
                         None) == 2
+
+
+def test_allreduce_argument_checks(lib):
+    """fp4_allreduce_sum_f32 validates before touching NCCL: no communicator,
+    a negative count, a misaligned buffer; an empty sum does nothing."""
+    comm = C.c_void_p(1 << 20)
+    assert lib.fp4_allreduce_sum_f32(None, C.c_void_p(1 << 21), 4, None) == 1
+    assert lib.fp4_allreduce_sum_f32(comm, C.c_void_p(1 << 21), -1, None) == 2
+    assert lib.fp4_allreduce_sum_f32(comm, C.c_void_p((1 << 21) + 2), 4, None) == 3
+    assert lib.fp4_allreduce_sum_f32(comm, None, 0, None) == 0
