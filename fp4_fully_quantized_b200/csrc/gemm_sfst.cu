@@ -16,9 +16,10 @@
 //   warps 4..11  epilogue: quadrant warp % 4, column half (warp - 4) / 4
 //   warp 12      TMA producer (A, B and the scale atoms into a 4-stage ring)
 //   warp 13      TMEM allocation and MMA issue
-// Barriers per stage: full (TMA landed) -> scales (4 stagers wrote TMEM) ->
-// empty (the MMAs that read the stage finished; tcgen05.commit).  All waits
-// are bounded.
+// Barriers per stage: atoms (the scale atoms landed) -> scales (4 stagers
+// wrote TMEM); full (the A and B tiles landed); the MMAs wait for both, and
+// empty (the MMAs that read the stage finished; tcgen05.commit) frees the stage
+// and its TMEM slot.  All waits are bounded.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -110,10 +111,11 @@ fp4_gemm_sfst_kernel(const __grid_constant__ CUtensorMap tmap_a,
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
   auto sf_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };
-  const uint32_t acc_full = bar0 + 8u * (3 * STAGES);
-  const uint32_t acc_empty = bar0 + 8u * (3 * STAGES + 1);
-  const uint32_t drain_bar = bar0 + 8u * (3 * STAGES + 2);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 3);
+  auto atoms_bar = [&](int s) { return bar0 + 8u * (3 * STAGES + s); };
+  const uint32_t acc_full = bar0 + 8u * (4 * STAGES);
+  const uint32_t acc_empty = bar0 + 8u * (4 * STAGES + 1);
+  const uint32_t drain_bar = bar0 + 8u * (4 * STAGES + 2);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 4 * STAGES + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -127,6 +129,7 @@ fp4_gemm_sfst_kernel(const __grid_constant__ CUtensorMap tmap_a,
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
       mbar_init(sf_bar(s), 4);
+      mbar_init(atoms_bar(s), 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, EPI_WARPS);
@@ -158,23 +161,27 @@ fp4_gemm_sfst_kernel(const __grid_constant__ CUtensorMap tmap_a,
           if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, p.status, 0x3100 + s)) { ok = false; break; }
           const int n_atoms = NV ? min(4, apr - kb * 4) : min(2, apr - kb * 2);
           const uint32_t atom_bytes = (uint32_t)n_atoms * 512u;
-          mbar_arrive_expect_tx(full_bar(s), A_BYTES + B_BYTES + atom_bytes * (b_hi ? 3u : 2u));
-          tma_load_2d(smem_u32(sA(s)), &tmap_a, full_bar(s), kb * (BK / 2), mb * BM);
-          tma_load_2d(smem_u32(sB(s)), &tmap_b, full_bar(s), kb * (BK / 2), nb * BN);
+          // scale atoms first, on their own barrier: the stagers move them into
+          // tensor memory while the operand tiles are still in flight
+          mbar_arrive_expect_tx(atoms_bar(s), atom_bytes * (b_hi ? 3u : 2u));
           const int atom0 = kb * (NV ? 4 : 2);
           bulk_load(smem_u32(sSFA(s)), p.a_sf + ((size_t)mb * apr + atom0) * 512, atom_bytes,
-                    full_bar(s));
+                    atoms_bar(s));
           bulk_load(smem_u32(sSFB(s)), p.b_sf + ((size_t)(2 * nb) * apr + atom0) * 512, atom_bytes,
-                    full_bar(s));
+                    atoms_bar(s));
           if (b_hi)
             bulk_load(smem_u32(sSFB(s) + 4 * 512), p.b_sf + ((size_t)(2 * nb + 1) * apr + atom0) * 512,
-                      atom_bytes, full_bar(s));
+                      atom_bytes, atoms_bar(s));
+          mbar_arrive_expect_tx(full_bar(s), A_BYTES + B_BYTES);
+          tma_load_2d(smem_u32(sA(s)), &tmap_a, full_bar(s), kb * (BK / 2), mb * BM);
+          tma_load_2d(smem_u32(sB(s)), &tmap_b, full_bar(s), kb * (BK / 2), nb * BN);
         }
       }
       if (it > 0) {
         const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0;
         for (uint32_t j = first; j < it; ++j) {
           volatile int no_abort = 0;
+          mbar_wait(atoms_bar(j % STAGES), (j / STAGES) & 1u, &no_abort, p.status, 0x3200 + j % STAGES);
           mbar_wait(full_bar(j % STAGES), (j / STAGES) & 1u, &no_abort, p.status, 0x3200 + j % STAGES);
         }
       }
@@ -192,7 +199,7 @@ fp4_gemm_sfst_kernel(const __grid_constant__ CUtensorMap tmap_a,
       for (int kb = 0; kb < k_blocks; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1u;
-        if (!warp_wait(full_bar(s), ph, abort_flag, p.status, 0x3300 + s, lane)) { ok = false; break; }
+        if (!warp_wait(atoms_bar(s), ph, abort_flag, p.status, 0x3300 + s, lane)) { ok = false; break; }
         uint32_t va[16], vb[32];
         const uint8_t* fa = sSFA(s) + lane * 16;
         const uint8_t* fb = sSFB(s) + lane * 16;
@@ -226,6 +233,7 @@ fp4_gemm_sfst_kernel(const __grid_constant__ CUtensorMap tmap_a,
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           if (!mbar_wait(sf_bar(s), ph, abort_flag, p.status, 0x3500 + s)) { ok = false; break; }
+          if (!mbar_wait(full_bar(s), ph, abort_flag, p.status, 0x3580 + s)) { ok = false; break; }
           tc_fence_after();
           const int n_mma = min(BK / MMA_K, (p.K - kb * BK) / MMA_K);
           const uint32_t t_sfa = tmem_base + TMEM_SF_BASE + s * TMEM_SF_STAGE;

@@ -13,6 +13,10 @@
 //   4  as 0, with the copies issued concurrently by a second warp (into a
 //      separate TMEM region) instead of by the MMA thread
 //   5  as 2, the same for the CTA pair
+//   6  as 0, with one K step's twelve copies (4 A atoms, 8 B atoms) issued
+//      together before its 4 MMAs, into five rotating 48-column slots: the
+//      order and tensor-memory layout a copy-fed GEMM would use
+//   7  as 6, for the CTA pair (tcgen05.cp.cta_group::2)
 // Operands are filled with pseudo-random codes and unit scales.  Waits are
 // bounded like the GEMM's.
 #include <cuda.h>
@@ -93,7 +97,7 @@ __device__ __forceinline__ uint32_t hash32(uint32_t x) {
   return x;
 }
 
-template <bool PAIR, bool WITH_CP, bool CP_WARP = false>
+template <bool PAIR, bool WITH_CP, bool CP_WARP = false, bool BATCH = false>
 __device__ void peak_body(int iters, uint32_t* status, uint8_t* base) {
   uint8_t* sA = base;
   uint8_t* sB = base + A_BYTES;
@@ -160,13 +164,29 @@ __device__ void peak_body(int iters, uint32_t* status, uint8_t* base) {
     const uint32_t idesc = make_idesc(256, PAIR ? 256 : 128, 0u, 0u, 0u);
     const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
     for (int i = 0; i < iters; ++i) {
+      // BATCH: this K step's slot (columns 256..495)
+      const uint32_t ks = tmem + 256 + 48 * (uint32_t)(i % 5);
+      if (BATCH) {
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          if (PAIR) tc_cp_pair_32x128b(ks + 4 * a, sf0);
+          else tc_cp_32x128b(ks + 4 * a, sf0);
+        }
+#pragma unroll
+        for (int a = 0; a < 8; ++a) {
+          if (PAIR) tc_cp_pair_32x128b(ks + 16 + 4 * a, sf1);
+          else tc_cp_32x128b(ks + 16 + 4 * a, sf1);
+        }
+      }
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         if (WITH_CP) cp_all();
         const uint64_t ad = smem_desc(a_base + kk * 32, 16, 1024, 2);
         const uint64_t bd = smem_desc(b_base + kk * 32, 16, 1024, 2);
-        if (PAIR) tc_mma_pair<true>(tmem, ad, bd, idesc, t_sfa, t_sfb, 1u);
-        else tc_mma<true>(tmem, ad, bd, idesc, t_sfa, t_sfb, 1u);
+        const uint32_t sfa = BATCH ? ks + 4 * kk : t_sfa;
+        const uint32_t sfb = BATCH ? ks + 16 + 8 * kk : t_sfb;
+        if (PAIR) tc_mma_pair<true>(tmem, ad, bd, idesc, sfa, sfb, 1u);
+        else tc_mma<true>(tmem, ad, bd, idesc, sfa, sfb, 1u);
       }
     }
     if (PAIR) tc_commit_pair(smem_u32(bar), 0x1);
@@ -183,19 +203,19 @@ __device__ void peak_body(int iters, uint32_t* status, uint8_t* base) {
   }
 }
 
-template <bool WITH_CP, bool CP_WARP>
+template <bool WITH_CP, bool CP_WARP, bool BATCH = false>
 __global__ void __launch_bounds__(128, 1) mma_peak_single(int iters, uint32_t* status) {
   extern __shared__ uint8_t sm[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm) + 1023) & ~uintptr_t(1023));
-  peak_body<false, WITH_CP, CP_WARP>(iters, status, base);
+  peak_body<false, WITH_CP, CP_WARP, BATCH>(iters, status, base);
 }
 
-template <bool WITH_CP, bool CP_WARP>
+template <bool WITH_CP, bool CP_WARP, bool BATCH = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1)
 mma_peak_pair(int iters, uint32_t* status) {
   extern __shared__ uint8_t sm[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm) + 1023) & ~uintptr_t(1023));
-  peak_body<true, WITH_CP, CP_WARP>(iters, status, base);
+  peak_body<true, WITH_CP, CP_WARP, BATCH>(iters, status, base);
 }
 
 }  // namespace
@@ -207,7 +227,7 @@ extern "C" fp4_status fp4_mma_rate(int32_t variant, int32_t iters, float* tflops
                                    void* ws, size_t ws_bytes, void* stream) {
   if (tflops_out == nullptr || ws == nullptr) return FP4_ERR_NULL;
   if (ws_bytes < sizeof(DeviceStatus)) return FP4_ERR_WORKSPACE;
-  if (variant < 0 || variant > 5 || iters <= 0) return FP4_ERR_SHAPE;
+  if (variant < 0 || variant > 7 || iters <= 0) return FP4_ERR_SHAPE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int grid = (sm_count() / 2) * 2;
   uint32_t* status = static_cast<uint32_t*>(ws);
@@ -223,7 +243,9 @@ extern "C" fp4_status fp4_mma_rate(int32_t variant, int32_t iters, float* tflops
       case 2: FP4_PEAK_LAUNCH((mma_peak_pair<false, false>)); break;
       case 3: FP4_PEAK_LAUNCH((mma_peak_pair<true, false>)); break;
       case 4: FP4_PEAK_LAUNCH((mma_peak_single<false, true>)); break;
-      default: FP4_PEAK_LAUNCH((mma_peak_pair<false, true>)); break;
+      case 5: FP4_PEAK_LAUNCH((mma_peak_pair<false, true>)); break;
+      case 6: FP4_PEAK_LAUNCH((mma_peak_single<false, false, true>)); break;
+      default: FP4_PEAK_LAUNCH((mma_peak_pair<false, false, true>)); break;
 #undef FP4_PEAK_LAUNCH
     }
     count_launches(1);
@@ -240,7 +262,7 @@ extern "C" fp4_status fp4_mma_rate(int32_t variant, int32_t iters, float* tflops
   cudaEventDestroy(e1);
   // flops: each CTA (single) or CTA pair issues iters * 4 MMAs of
   // 128x256x64 (single) or 256x256x64 (pair)
-  const bool pair = variant == 2 || variant == 3 || variant == 5;
+  const bool pair = variant == 2 || variant == 3 || variant == 5 || variant == 7;
   const double per_mma = pair ? 2.0 * 256 * 256 * 64 : 2.0 * 128 * 256 * 64;
   const double issuers = pair ? grid / 2 : grid;
   *tflops_out = (float)(issuers * 4.0 * iters * per_mma / (ms * 1e-3) / 1e12);

@@ -343,12 +343,14 @@ const char* fp4_status_str(int32_t status);
 int32_t fp4_abi_version(void);
 
 /* Tensor-core rate microbenchmark (synchronises `stream`): one persistent CTA
- * (variants 0, 1, 4) or CTA pair (2, 3, 5) per SM issues `iters` x 4
+ * (variants 0, 1, 4, 6) or CTA pair (2, 3, 5, 7) per SM issues `iters` x 4
  * back-to-back block-scaled NVFP4 MMAs (128x256x64, or 256x256x64 for a
  * pair) on operands resident in shared memory; variants 1 and 3 add, from the
  * MMA thread, the three scale-factor copies into tensor memory that one MMA
  * of a GEMM K step needs; variants 4 and 5 issue the same copies from a
- * second warp concurrently with the MMAs.  Writes the
+ * second warp concurrently with the MMAs; variants 6 and 7 issue a K step's
+ * twelve copies together before its four MMAs, into rotating slots.  Any other
+ * variant, or iters <= 0, returns FP4_ERR_SHAPE.  Writes the
  * achieved TFLOP/s: what the tensor pipe sustains with and without the
  * scale-factor traffic, the context for the GEMM's rate ("FP4" page,
  * Hardware: FP4 on fifth-generation Tensor Cores). */
