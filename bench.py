@@ -43,7 +43,7 @@ FP4_PER_BF16 = 4.0          # nominal dense FP4 / dense BF16 tensor throughput (
 # figures); multiplied by the step's average FLOPs per GEMM launch it is
 # `roofline.traffic`.  None whenever the GEMM kernel changes until
 # re-measured.
-GEMM_DRAM_BYTES_PER_FLOP = 3.022e-4
+GEMM_DRAM_BYTES_PER_FLOP = 3.006e-4
 # Algorithmic bytes per element of one quantize call producing row-wise and
 # transposed outputs with an in-kernel amax: amax read 2 B + encode read 2 B
 # + two outputs of (0.5 B codes + 1/16 B scales).
