@@ -982,9 +982,61 @@ def run_formats(device, seed=0, rows_checked=128, M=M_TOKENS):
     return out
 
 
+def _time(fn, steps, warmup):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps
+
+
+def run_gemm_vendor(F, qa, qb, y, ws, args):
+    """Comparison only, never the library's path: the vendor's block-scaled
+    NVFP4 GEMM (cuBLASLt through torch.nn.functional.scaled_mm) on the very
+    operand bytes fp4_gemm reads (E2M1 codes, E4M3 block scales in the
+    128-row x 4-block atom layout, FP32 tensor scales), BF16 out, both timed
+    the same way; the two products are compared element by element."""
+    import torch.nn.functional as Fn
+    M, N, K = qa.rows, qb.rows, qa.cols
+    fp4 = torch.float4_e2m1fn_x2
+    a = qa.codes.view(M, K // 2).view(fp4)
+    b = qb.codes.view(N, K // 2).view(fp4).t()
+    sa = qa.scales_mma.view(torch.float8_e4m3fn)
+    sb = qb.scales_mma.view(torch.float8_e4m3fn)
+    ST, SW = Fn.ScalingType, Fn.SwizzleType
+    vend = lambda: Fn.scaled_mm(a, b, [sa, qa.s_dec], [ST.BlockWise1x16, ST.TensorWise],
+                                [sb, qb.s_dec], [ST.BlockWise1x16, ST.TensorWise],
+                                swizzle_a=[SW.SWIZZLE_32_4_4, SW.NO_SWIZZLE],
+                                swizzle_b=[SW.SWIZZLE_32_4_4, SW.NO_SWIZZLE],
+                                output_dtype=torch.bfloat16)
+    ours = lambda: F.fp4_gemm(qa, qb, y, ws=ws)
+    ms_v = _time(vend, args.steps, args.warmup)
+    ms_o = _time(ours, args.steps, args.warmup)
+    yv = vend()
+    ours()
+    torch.cuda.synchronize()
+    assert ws.status() == 0
+    d = (yv.float() - y.float()).abs()
+    fl = 2.0 * M * N * K / 1e12
+    return {"case": "gemm_vendor", "m": M, "n": N, "k": K, "unit": "TFLOP/s",
+            "vendor": {"ms": round(ms_v, 4), "rate": round(fl / (ms_v * 1e-3), 1),
+                       "kernel": "torch.nn.functional.scaled_mm (cuBLASLt), NVFP4 two-level"},
+            "ours": {"ms": round(ms_o, 4), "rate": round(fl / (ms_o * 1e-3), 1)},
+            "ratio_ours_to_vendor": round(ms_v / ms_o, 3),
+            "bf16_equal_frac": round(float((yv == y).float().mean().item()), 4),
+            "max_abs_diff_over_max": float(d.max().item() / max(float(y.float().abs().max().item()), 1e-30))}
+
+
 def run_case(args, device):
     """A single kernel family on one small problem (for profiler captures):
     --case gemm: NVFP4 fprop-style GEMM [m, k] x [n, k]^T, BF16 out;
+    --case gemm_vendor: the same operands through the vendor's NVFP4 GEMM,
+    timed beside fp4_gemm (comparison only);
     --case quant: NVFP4 row-wise RTN + transposed SR of a [m, k] tensor;
     --case quant_sr: both outputs stochastically rounded (the dY quantization);
     --case gemm_quant / gemm_then_quant: the GEMM with its result encoded to
@@ -1019,6 +1071,8 @@ def run_case(args, device):
                         device=device)
         qy = F.QTensor.empty(M, N, device=device, logical_scales=False)
         y_amax = torch.ones(1, dtype=torch.float32, device=device)   # supplied (delayed) amax
+        if args.case == "gemm_vendor":
+            return run_gemm_vendor(F, qa, qb, y, ws, args)
         if args.case == "gemm_quant":          # result encoded to NVFP4 in the epilogue
             fn = lambda: F.fp4_gemm_quant(qa, qb, qy, y_amax, ws=ws)
         elif args.case == "gemm_then_quant":   # BF16 result, then the quantizer
@@ -1043,8 +1097,8 @@ def run_case(args, device):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--case", choices=["gemm", "gemm_quant", "gemm_then_quant", "quant", "quant_sr",
-                                       "sweep", "swiglu", "formats"], default=None,
+    ap.add_argument("--case", choices=["gemm", "gemm_vendor", "gemm_quant", "gemm_then_quant", "quant",
+                                       "quant_sr", "sweep", "swiglu", "formats"], default=None,
                     help="time one kernel family on one problem (profiling), or the "
                          "quantizer sweep over 2^n elements")
     ap.add_argument("--rounds", default=None,

@@ -1,0 +1,54 @@
+"""fp4_gemm against an independent implementation: the vendor's block-scaled
+NVFP4 GEMM (cuBLASLt through torch.nn.functional.scaled_mm), given the very
+operand bytes fp4_gemm reads (E2M1 codes, E4M3 block scales in the 128-row x
+4-block atom layout, FP32 tensor scales).  Both accumulate in FP32 and round
+once to BF16, so on these shapes the two BF16 products are equal element for
+element.  The vendor kernel is used here and in `bench.py --case gemm_vendor`
+only, as a cross-check and a rate to compare with, never on the library's
+path."""
+import pytest
+import torch
+
+import fqt_synth as S
+
+pytestmark = pytest.mark.gpu
+
+Fn = torch.nn.functional
+
+
+def _vendor(qa, qb):
+    M, N, K = qa.rows, qb.rows, qa.cols
+    fp4 = torch.float4_e2m1fn_x2
+    ST, SW = Fn.ScalingType, Fn.SwizzleType
+    return Fn.scaled_mm(qa.codes.view(M, K // 2).view(fp4), qb.codes.view(N, K // 2).view(fp4).t(),
+                        [qa.scales_mma.view(torch.float8_e4m3fn), qa.s_dec],
+                        [ST.BlockWise1x16, ST.TensorWise],
+                        [qb.scales_mma.view(torch.float8_e4m3fn), qb.s_dec],
+                        [ST.BlockWise1x16, ST.TensorWise],
+                        swizzle_a=[SW.SWIZZLE_32_4_4, SW.NO_SWIZZLE],
+                        swizzle_b=[SW.SWIZZLE_32_4_4, SW.NO_SWIZZLE],
+                        output_dtype=torch.bfloat16)
+
+
+@pytest.mark.parametrize("M,N,K,w_block", [(256, 512, 1024, "1d"), (384, 640, 512, "2d"),
+                                           (1024, 768, 4096, "2d"), (128, 384, 320, "1d")])
+def test_fp4_gemm_equals_vendor_nvfp4_gemm(gpu_lib, M, N, K, w_block):
+    if not hasattr(Fn, "scaled_mm") or not hasattr(torch, "float4_e2m1fn_x2"):
+        pytest.skip("this torch has no NVFP4 scaled_mm")
+    F = gpu_lib
+    dev = torch.device("cuda", 0)
+    blk = F.BLOCK_2D if w_block == "2d" else F.BLOCK_1D
+    x = S.student_t_channels(M, K, seed=M + K)[0].to(dev)
+    w = S.normal((N, K), 0.02, seed=N + K).to(dev)
+    qa = F.QTensor.empty(M, K, device=dev, logical_scales=False)
+    qb = F.QTensor.empty(N, K, F.NVFP4, blk, device=dev, logical_scales=False)
+    ws = F.Workspace(M, N, K, device=dev)
+    F.fp4_quantize(x, qa, ws=ws)
+    F.fp4_quantize(w, qb, block=blk, ws=ws)
+    y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=dev)
+    F.fp4_gemm(qa, qb, y, ws=ws)
+    yv = _vendor(qa, qb)
+    torch.cuda.synchronize()
+    assert ws.status() == 0
+    assert torch.isfinite(y).all()
+    assert torch.equal(y, yv)
