@@ -1008,23 +1008,33 @@ def _time(fn, steps, warmup):
 
 def run_gemm_vendor(F, qa, qb, y, ws, args):
     """Comparison only, never the library's path: the vendor's block-scaled
-    NVFP4 GEMM (cuBLASLt through torch.nn.functional.scaled_mm) on the very
-    operand bytes fp4_gemm reads (E2M1 codes, E4M3 block scales in the
-    128-row x 4-block atom layout, FP32 tensor scales), BF16 out, both timed
-    the same way; the two products are compared element by element."""
+    FP4 GEMM (cuBLASLt through torch.nn.functional.scaled_mm) on the very
+    operand bytes fp4_gemm reads (E2M1 codes; E4M3 block scales and FP32
+    tensor scales for NVFP4, E8M0 block scales for MXFP4; scales in the
+    128-row x 4-block atom layout), BF16 out, both timed the same way; the two
+    products are compared element by element."""
     import torch.nn.functional as Fn
     M, N, K = qa.rows, qb.rows, qa.cols
     fp4 = torch.float4_e2m1fn_x2
     a = qa.codes.view(M, K // 2).view(fp4)
     b = qb.codes.view(N, K // 2).view(fp4).t()
-    sa = qa.scales_mma.view(torch.float8_e4m3fn)
-    sb = qb.scales_mma.view(torch.float8_e4m3fn)
     ST, SW = Fn.ScalingType, Fn.SwizzleType
-    vend = lambda: Fn.scaled_mm(a, b, [sa, qa.s_dec], [ST.BlockWise1x16, ST.TensorWise],
-                                [sb, qb.s_dec], [ST.BlockWise1x16, ST.TensorWise],
-                                swizzle_a=[SW.SWIZZLE_32_4_4, SW.NO_SWIZZLE],
-                                swizzle_b=[SW.SWIZZLE_32_4_4, SW.NO_SWIZZLE],
-                                output_dtype=torch.bfloat16)
+    if qa.fmt == F.MXFP4:             # E8M0 1x32 block scales, tensor scale 1
+        sa = qa.scales_mma.view(torch.float8_e8m0fnu)
+        sb = qb.scales_mma.view(torch.float8_e8m0fnu)
+        vend = lambda: Fn.scaled_mm(a, b, sa, ST.BlockWise1x32, sb, ST.BlockWise1x32,
+                                    swizzle_a=SW.SWIZZLE_32_4_4, swizzle_b=SW.SWIZZLE_32_4_4,
+                                    output_dtype=torch.bfloat16)
+        recipe = "MXFP4"
+    else:
+        sa = qa.scales_mma.view(torch.float8_e4m3fn)
+        sb = qb.scales_mma.view(torch.float8_e4m3fn)
+        vend = lambda: Fn.scaled_mm(a, b, [sa, qa.s_dec], [ST.BlockWise1x16, ST.TensorWise],
+                                    [sb, qb.s_dec], [ST.BlockWise1x16, ST.TensorWise],
+                                    swizzle_a=[SW.SWIZZLE_32_4_4, SW.NO_SWIZZLE],
+                                    swizzle_b=[SW.SWIZZLE_32_4_4, SW.NO_SWIZZLE],
+                                    output_dtype=torch.bfloat16)
+        recipe = "NVFP4 two-level"
     ours = lambda: F.fp4_gemm(qa, qb, y, ws=ws)
     ms_v = _time(vend, args.steps, args.warmup)
     ms_o = _time(ours, args.steps, args.warmup)
@@ -1036,7 +1046,7 @@ def run_gemm_vendor(F, qa, qb, y, ws, args):
     fl = 2.0 * M * N * K / 1e12
     return {"case": "gemm_vendor", "m": M, "n": N, "k": K, "unit": "TFLOP/s",
             "vendor": {"ms": round(ms_v, 4), "rate": round(fl / (ms_v * 1e-3), 1),
-                       "kernel": "torch.nn.functional.scaled_mm (cuBLASLt), NVFP4 two-level"},
+                       "kernel": "torch.nn.functional.scaled_mm (cuBLASLt), " + recipe},
             "ours": {"ms": round(ms_o, 4), "rate": round(fl / (ms_o * 1e-3), 1)},
             "ratio_ours_to_vendor": round(ms_v / ms_o, 3),
             "bf16_equal_frac": round(float((yv == y).float().mean().item()), 4),
@@ -1074,6 +1084,13 @@ def run_case(args, device):
         units, unit = M * K * bpe / 1e9, "GB/s"
     else:
         w = S.normal((N, K), 0.02, seed=2).to(device)
+        if args.case == "gemm_vendor" and args.fmt == "mxfp4":
+            qa = F.QTensor.empty(M, K, F.MXFP4, device=device, logical_scales=False)
+            qb = F.QTensor.empty(N, K, F.MXFP4, device=device, logical_scales=False)
+            F.fp4_quantize(x, qa, fmt=F.MXFP4, ws=ws)
+            F.fp4_quantize(w, qb, fmt=F.MXFP4, ws=ws)
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+            return run_gemm_vendor(F, qa, qb, y, ws, args)
         qb = F.QTensor.empty(N, K, F.NVFP4, F.BLOCK_2D, device=device, logical_scales=False)
         qbt = F.QTensor.empty(K, N, F.NVFP4, F.BLOCK_2D, device=device, logical_scales=False)
         F.fp4_quantize(x, qa, ws=ws)
