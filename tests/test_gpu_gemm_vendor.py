@@ -32,7 +32,8 @@ def _vendor(qa, qb):
 
 
 @pytest.mark.parametrize("M,N,K,w_block", [(256, 512, 1024, "1d"), (384, 640, 512, "2d"),
-                                           (1024, 768, 4096, "2d"), (128, 384, 320, "1d")])
+                                           (1024, 768, 4096, "2d"), (128, 384, 320, "1d"),
+                                           (8192, 4096, 8192, "2d")])
 def test_fp4_gemm_equals_vendor_nvfp4_gemm(gpu_lib, M, N, K, w_block):
     if not hasattr(Fn, "scaled_mm") or not hasattr(torch, "float4_e2m1fn_x2"):
         pytest.skip("this torch has no NVFP4 scaled_mm")
