@@ -1,12 +1,14 @@
 """fp4_gemm against an independent implementation: the vendor's block-scaled
 NVFP4 GEMM (cuBLASLt through torch.nn.functional.scaled_mm), given the very
 operand bytes fp4_gemm reads (E2M1 codes, E4M3 block scales in the 128-row x
-4-block atom layout, FP32 tensor scales).  Both accumulate in FP32 and round
-once to BF16, so on these shapes the two BF16 products are equal element for
-element.  The same holds for MXFP4 (E8M0 1x32 block scales, tensor scale 1)
-against the vendor's MX recipe.  The vendor kernel is used here and in
-`bench.py --case gemm_vendor` only, as a cross-check and a rate to compare
-with, never on the library's path."""
+4-block atom layout, FP32 tensor scales), and the same for MXFP4 (E8M0 1x32
+block scales, tensor scale 1) against the vendor's MX recipe.  Both
+accumulate in FP32 and round once to BF16; with the kernels the vendor picks
+on B200 the two products are identical element for element (reported), and
+the test requires agreement within one BF16 rounding of the product, since
+which vendor kernel runs (and its accumulation order) is the vendor's choice.
+The vendor kernel is used here and in `bench.py --case gemm_vendor` only, as
+a cross-check and a rate to compare with, never on the library's path."""
 import pytest
 import torch
 
@@ -15,6 +17,19 @@ import fqt_synth as S
 pytestmark = pytest.mark.gpu
 
 Fn = torch.nn.functional
+
+
+def _agree(y, yv):
+    """Equal, or apart by at most one BF16 unit (2^-7 of each element) plus an
+    absolute floor of 2^-12 of the largest output for elements that cancel:
+    what a different FP32 accumulation order can change.  A wrong product
+    (operand, scale or layout) is off by far more."""
+    if torch.equal(y, yv):
+        print("bit-identical")
+        return
+    a, b = y.float(), yv.float()
+    tol = torch.maximum(a.abs(), b.abs()) * 2.0 ** -7 + a.abs().max() * 2.0 ** -12
+    assert bool(((a - b).abs() <= tol).all())
 
 
 def _vendor(qa, qb):
@@ -53,7 +68,7 @@ def test_fp4_gemm_equals_vendor_nvfp4_gemm(gpu_lib, M, N, K, w_block):
     torch.cuda.synchronize()
     assert ws.status() == 0
     assert torch.isfinite(y).all()
-    assert torch.equal(y, yv)
+    _agree(y, yv)
 
 
 def _vendor_mx(qa, qb):
@@ -89,4 +104,4 @@ def test_fp4_gemm_equals_vendor_mxfp4_gemm(gpu_lib, M, N, K, quest):
     torch.cuda.synchronize()
     assert ws.status() == 0
     assert torch.isfinite(y).all()
-    assert torch.equal(y, yv)
+    _agree(y, yv)
